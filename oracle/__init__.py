@@ -1,0 +1,30 @@
+"""CPU oracle for the FP8 W8A8 linear path — TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, obviously correct NumPy restatement of what the CUDA path
+computes, used to check it.  Only the tests, the smoke check and the CPU
+baseline leg of the benchmark may import this package; the product path never
+does, and this package imports nothing from the product package.
+
+Sources (two web pages describing the same method):
+  [P1] "Quantized Inference for OneRec-V2：生成式推荐开始直接吃 LLM 量化栈",
+       section 关键证据 — weights quantized offline per output channel,
+       activations quantized per token at run time, FP8 tensor-core matmul
+       with FP32 accumulation, output cast back to FP16.
+  [P2] "FP8量化在生成式推荐系统OneRec-V2中的优化实践", §1.2 (FP8 range ±448),
+       §2.2 (E4M3 format; per-token dynamic scale computed as
+       max_code / max|x| with an eps floor), §2.3 (FP8 multiply + FP32
+       accumulate + FP16 output).
+
+Where the pages leave a step open the reading taken is stated beside the code
+(rounding: round-to-nearest-even, saturating to ±448; eps = 1e-12; scale
+stored as amax/448 and codes produced with one fp32 multiply by 448/amax).
+
+Every function here is pinned by tests against closed forms, hand-worked
+rows, a library cast routine and brute force; none is "parity unpinned".
+"""
+from .e4m3 import E4M3_MAX, e4m3_decode, e4m3_encode
+from .quant import EPS, quant_rows
+from .linear import linear_ref, moe_ref, linear_f64_unquantized
+
+__all__ = ["E4M3_MAX", "e4m3_decode", "e4m3_encode", "EPS", "quant_rows",
+           "linear_ref", "moe_ref", "linear_f64_unquantized"]

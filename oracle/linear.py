@@ -1,0 +1,57 @@
+"""FP8 W8A8 linear and MoE grouped linear, double-accumulated.
+
+[P1 关键证据, steps 3-4; P2 §2.3]: the matmul multiplies FP8 operands and
+accumulates in at least FP32, then the result is brought back to FP16 before
+the next layer; the dequantization uses the per-token scale s_x[m] and the
+per-channel scale s_w[n].  Here the products and sums are taken in float64
+(exact products, near-exact sums) so the oracle is at least as accurate as
+any FP32 accumulation order:
+
+    P[m,n] = sum_k dec(Xq[m,k]) * dec(Wq[n,k])          (float64)
+    Y[m,n] = fp16_rne( (P[m,n] * s_x[m]) * s_w[n] )     (float64 -> float16)
+
+No bias term (the pages name none).  The float64 -> float16 cast is NumPy's
+direct, correctly rounded conversion (round half to even, overflow to inf).
+
+MoE [P1 关键证据 item 2: the sparse MoE grouped GEMM]: rows are grouped by
+expert, rows offsets[e]..offsets[e+1] use expert e's weights and scales.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .e4m3 import e4m3_decode
+
+
+def linear_ref(Xq, s_x, Wq, s_w) -> np.ndarray:
+    """Xq uint8 [M,K], s_x f32 [M], Wq uint8 [N,K], s_w f32 [N] -> float16 [M,N]."""
+    Dx = e4m3_decode(Xq)
+    Dw = e4m3_decode(Wq)
+    P = Dx @ Dw.T
+    Y = (P * np.asarray(s_x, dtype=np.float64)[:, None]) * np.asarray(s_w, dtype=np.float64)[None, :]
+    return Y.astype(np.float16)
+
+
+def moe_ref(Xq, s_x, offsets, Wq, s_w) -> np.ndarray:
+    """Grouped linear.
+
+    Xq uint8 [R,K] (rows in expert order), s_x f32 [R], offsets int [E+1]
+    with offsets[0] = 0 and offsets[E] = R, Wq uint8 [E,N,K], s_w f32 [E,N]
+    -> float16 [R,N].  Empty groups produce no rows.
+    """
+    offsets = np.asarray(offsets, dtype=np.int64)
+    E, N, _ = np.asarray(Wq).shape
+    R = np.asarray(Xq).shape[0]
+    if offsets.shape != (E + 1,) or offsets[0] != 0 or offsets[-1] != R or np.any(np.diff(offsets) < 0):
+        raise ValueError("offsets must be non-decreasing, start at 0 and end at the row count")
+    Y = np.zeros((R, N), dtype=np.float16)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            Y[lo:hi] = linear_ref(Xq[lo:hi], s_x[lo:hi], Wq[e], s_w[e])
+    return Y
+
+
+def linear_f64_unquantized(X, W) -> np.ndarray:
+    """X @ W^T in float64 on the original (unquantized) values, for error-bound pins."""
+    return np.asarray(X, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T

@@ -1,0 +1,146 @@
+"""Pins for the oracle's FP8 linear and MoE grouped linear.
+
+'Quantized Inference for OneRec-V2' (关键证据 steps 3-4) and
+'FP8量化在生成式推荐系统OneRec-V2中的优化实践' (§2.3): FP8 products, FP32 (here
+FP64) accumulation, per-token x per-channel dequantization, FP16 output.
+
+Pins:
+  * exactness: when every row's amax is 448*2^j and every entry is an E4M3
+    value times 2^j, quantization loses nothing and the result must equal
+    fp16(X @ W^T) computed in float64 directly from the fp16 inputs, bit for bit;
+  * brute force: on tiny random inputs the result stays within the analytic
+    quantization error bound of the unquantized float64 product;
+  * MoE: explicit per-row loops over expert groups, and the single-expert case.
+"""
+import numpy as np
+import pytest
+
+from oracle import e4m3_decode, linear_f64_unquantized, linear_ref, moe_ref, quant_rows
+
+
+FINITE_POS = e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))   # 0 .. 448
+
+
+def exact_matrix(rng, rows, cols, j):
+    """Entries = random E4M3 value * 2^j with random sign; each row holds one ±448*2^j."""
+    v = rng.choice(FINITE_POS, size=(rows, cols)) * rng.choice([-1.0, 1.0], size=(rows, cols))
+    where = rng.integers(0, cols, rows)
+    v[np.arange(rows), where] = 448.0 * rng.choice([-1.0, 1.0], size=rows)
+    m = (v * 2.0 ** j).astype(np.float16)
+    assert np.all(m.astype(np.float64) == v * 2.0 ** j)     # representable in fp16
+    return m
+
+
+@pytest.mark.parametrize("M,N,K,jx,jw", [(7, 5, 64, -4, -6), (33, 17, 96, -2, -8), (1, 64, 256, -3, -5)])
+def test_exactness_case(M, N, K, jx, jw):
+    rng = np.random.default_rng(M * 1000 + N)
+    X = exact_matrix(rng, M, K, jx)
+    W = exact_matrix(rng, N, K, jw)
+    Xq, sx = quant_rows(X)
+    Wq, sw = quant_rows(W)
+    assert np.all(sx == np.float32(2.0 ** jx)) and np.all(sw == np.float32(2.0 ** jw))
+    Y = linear_ref(Xq, sx, Wq, sw)
+    expect = (X.astype(np.float64) @ W.astype(np.float64).T).astype(np.float16)
+    np.testing.assert_array_equal(Y.view(np.uint16), expect.view(np.uint16))
+
+
+def quant_error_bound(X, W, sx, sw, Y):
+    """Analytic bound on |Y - X W^T| for the FP8 W8A8 linear.
+
+    Per element x: |dequant(x) - x| <= dx = max(2^-4 |x|, 2^-10 s) (3-bit
+    mantissa half-ulp; subnormal half-step 2^-10 scaled by s), plus fp32
+    rounding slack of the scale and product steps.  Summing products:
+    |sum xhat*what - sum x*w| <= sum (|x|+dx)(|w|+dw) - |x||w|; then one
+    fp16 rounding (half-ulp <= 2^-11 |y| for normals, 2^-25 below).
+    """
+    xa = np.abs(X.astype(np.float64))
+    wa = np.abs(W.astype(np.float64))
+    dx = np.maximum(2.0 ** -4 * xa, 2.0 ** -10 * sx.astype(np.float64)[:, None]) * (1 + 2.0 ** -18) + xa * 2.0 ** -20
+    dw = np.maximum(2.0 ** -4 * wa, 2.0 ** -10 * sw.astype(np.float64)[:, None]) * (1 + 2.0 ** -18) + wa * 2.0 ** -20
+    prod = (xa + dx) @ (wa + dw).T - xa @ wa.T
+    y = np.abs(Y.astype(np.float64))
+    return prod * (1 + 2.0 ** -40) + 2.0 ** -10 * y + 2.0 ** -24
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_brute_force_error_bound(seed):
+    rng = np.random.default_rng(100 + seed)
+    M, N, K = rng.integers(1, 17, 3)
+    X = (rng.standard_normal((M, K)) * np.exp(rng.uniform(-3, 3, (M, 1)))).astype(np.float16)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+    Xq, sx = quant_rows(X)
+    Wq, sw = quant_rows(W)
+    Y = linear_ref(Xq, sx, Wq, sw)
+    exact = linear_f64_unquantized(X, W)
+    err = np.abs(Y.astype(np.float64) - exact)
+    assert np.all(err <= quant_error_bound(X, W, sx, sw, Y))
+
+
+def test_bound_is_not_vacuous():
+    # The bound is tight enough to catch a transposed or dropped scale.
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((8, 32)).astype(np.float16)
+    W = (rng.standard_normal((8, 32)) * np.linspace(0.01, 0.5, 8)[:, None]).astype(np.float16)
+    Xq, sx = quant_rows(X)
+    Wq, sw = quant_rows(W)
+    exact = linear_f64_unquantized(X, W)
+    wrong = linear_ref(Xq, sx, Wq, sw[::-1].copy())
+    assert np.any(np.abs(wrong.astype(np.float64) - exact) > quant_error_bound(X, W, sx, sw, wrong))
+
+
+def test_zero_rows_and_columns():
+    X = np.zeros((3, 32), np.float16)
+    X[1] = 1.0
+    W = np.ones((4, 32), np.float16)
+    W[2] = 0
+    Xq, sx = quant_rows(X)
+    Wq, sw = quant_rows(W)
+    Y = linear_ref(Xq, sx, Wq, sw).astype(np.float64)
+    assert np.all(Y[0] == 0) and np.all(Y[2] == 0) and np.all(Y[:, 2] == 0)
+    assert Y[1, 0] == 32.0
+
+
+def _moe_loop(X, offsets, W):
+    """Per-row pure restatement with unquantized float64 inputs."""
+    out = np.zeros((X.shape[0], W.shape[1]))
+    for e in range(W.shape[0]):
+        for r in range(int(offsets[e]), int(offsets[e + 1])):
+            for n in range(W.shape[1]):
+                out[r, n] = float(np.dot(X[r].astype(np.float64), W[e, n].astype(np.float64)))
+    return out
+
+
+def test_moe_exact_groups_loop():
+    rng = np.random.default_rng(4)
+    E, N, K = 5, 6, 32
+    counts = [3, 0, 1, 4, 0]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    X = exact_matrix(rng, R, K, -3)
+    W = np.stack([exact_matrix(rng, N, K, -7) for _ in range(E)])
+    Xq, sx = quant_rows(X)
+    Wq, sw = quant_rows(W.reshape(E * N, K))
+    Y = moe_ref(Xq, sx, offsets, Wq.reshape(E, N, K), sw.reshape(E, N))
+    expect = _moe_loop(X, offsets, W).astype(np.float16)
+    np.testing.assert_array_equal(Y.view(np.uint16), expect.view(np.uint16))
+
+
+def test_moe_single_expert_is_linear():
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((20, 48)).astype(np.float16)
+    W = (rng.standard_normal((12, 48)) * 0.02).astype(np.float16)
+    Xq, sx = quant_rows(X)
+    Wq, sw = quant_rows(W)
+    Y1 = moe_ref(Xq, sx, np.array([0, 20], np.int32), Wq[None], sw[None])
+    exact = linear_f64_unquantized(X, W)
+    assert np.all(np.abs(Y1.astype(np.float64) - exact) <= quant_error_bound(X, W, sx, sw, Y1))
+
+
+def test_moe_rejects_bad_offsets():
+    Xq = np.zeros((4, 16), np.uint8)
+    sx = np.ones(4, np.float32)
+    Wq = np.zeros((2, 8, 16), np.uint8)
+    sw = np.ones((2, 8), np.float32)
+    for bad in ([0, 3, 2], [1, 2, 4], [0, 2, 5]):
+        with pytest.raises(ValueError):
+            moe_ref(Xq, sx, np.array(bad, np.int32), Wq, sw)

@@ -1,1 +1,127 @@
-"""B200-native FP8 W8A8 linear layers (binding filled in below)."""
+"""B200-native FP8 W8A8 linear layers (per-channel weights, per-token
+dynamic activations, FP8 tensor-core GEMM with FP32 accumulation and a fused
+dequantize + FP16 epilogue; dense and MoE grouped).
+
+The compute runs in libfp8q.so (hand-written sm_100a kernels behind a C ABI,
+include/fp8q.h).  This module only marshals torch tensors into that ABI:
+PyTorch provides device memory and streams.  There is no CPU fallback; a
+missing library raises ImportError at the first call.
+
+    Xq, s_x = quantize_rows_dynamic(X)          # X fp16 [M,K] on cuda
+    Wq, s_w = quantize_weight_per_channel(W)    # offline, W fp16 [N,K]
+    Y = linear(Xq, s_x, Wq, s_w)                # fp16 [M,N]
+    Y = moe_grouped_linear(Xq, s_x, offsets, Wq_e, s_w_e)
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+from ._lib import Fp8qError, check, lib
+
+__all__ = [
+    "Fp8qError", "lib", "quantize_rows_dynamic", "quantize_weight_per_channel", "linear",
+    "moe_grouped_linear", "quantized_linear", "e4m3_encode_f32", "device_error",
+]
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _need(t: torch.Tensor, dtype, name: str, ndim: int | None = None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
+
+
+def quantize_rows_dynamic(X: torch.Tensor, out: tuple | None = None):
+    """Per-token dynamic E4M3 quantization: fp16 [M,K] -> (uint8 [M,K], fp32 [M])."""
+    _need(X, torch.float16, "X", 2)
+    M, K = X.shape
+    Xq, s = out if out is not None else (
+        torch.empty((M, K), dtype=torch.uint8, device=X.device),
+        torch.empty((M,), dtype=torch.float32, device=X.device))
+    check(_lib.fp8q_quantize_rows_dynamic(X.data_ptr(), M, K, Xq.data_ptr(), s.data_ptr(), _stream(X)),
+          "fp8q_quantize_rows_dynamic")
+    return Xq, s
+
+
+def quantize_weight_per_channel(W: torch.Tensor):
+    """Offline per-output-channel E4M3 quantization: fp16 [N,K] or [E,N,K]."""
+    _need(W, torch.float16, "W")
+    if W.dim() not in (2, 3):
+        raise ValueError("W must be [N,K] or [E,N,K]")
+    K = W.shape[-1]
+    rows = W.numel() // K
+    Wq = torch.empty(W.shape, dtype=torch.uint8, device=W.device)
+    s = torch.empty(W.shape[:-1], dtype=torch.float32, device=W.device)
+    check(_lib.fp8q_quantize_weight_per_channel(W.data_ptr(), rows, K, Wq.data_ptr(), s.data_ptr(), _stream(W)),
+          "fp8q_quantize_weight_per_channel")
+    return Wq, s
+
+
+def linear(Xq: torch.Tensor, s_x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
+           out: torch.Tensor | None = None) -> torch.Tensor:
+    """FP8 W8A8 linear with fused dequantization: fp16 [M,N]."""
+    _need(Xq, torch.uint8, "Xq", 2)
+    _need(Wq, torch.uint8, "Wq", 2)
+    _need(s_x, torch.float32, "s_x", 1)
+    _need(s_w, torch.float32, "s_w", 1)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or s_x.shape[0] != M or s_w.shape[0] != N:
+        raise ValueError("shape mismatch")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=Xq.device)
+    check(_lib.fp8q_linear(Xq.data_ptr(), s_x.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K, Y.data_ptr(),
+                           _stream(Xq)), "fp8q_linear")
+    return Y
+
+
+def quantized_linear(X: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor) -> torch.Tensor:
+    """fp16 activations in, fp16 out: per-token quantization then the FP8 linear."""
+    Xq, s_x = quantize_rows_dynamic(X)
+    return linear(Xq, s_x, Wq, s_w)
+
+
+def moe_grouped_linear(Xq: torch.Tensor, s_x: torch.Tensor, offsets: torch.Tensor, Wq: torch.Tensor,
+                       s_w: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Expert-grouped FP8 linear.  offsets: int32 [E+1] on the device."""
+    _need(Xq, torch.uint8, "Xq", 2)
+    _need(s_x, torch.float32, "s_x", 1)
+    _need(offsets, torch.int32, "offsets", 1)
+    _need(Wq, torch.uint8, "Wq", 3)
+    _need(s_w, torch.float32, "s_w", 2)
+    rows, K = Xq.shape
+    E, N, K2 = Wq.shape
+    if K2 != K or offsets.shape[0] != E + 1 or tuple(s_w.shape) != (E, N) or s_x.shape[0] != rows:
+        raise ValueError("shape mismatch")
+    Y = out if out is not None else torch.empty((rows, N), dtype=torch.float16, device=Xq.device)
+    check(_lib.fp8q_moe_grouped_linear(Xq.data_ptr(), s_x.data_ptr(), offsets.data_ptr(), E, rows, Wq.data_ptr(),
+                                       s_w.data_ptr(), N, K, Y.data_ptr(), _stream(Xq)),
+          "fp8q_moe_grouped_linear")
+    return Y
+
+
+def e4m3_encode_f32(x: torch.Tensor) -> torch.Tensor:
+    """The device E4M3 cast alone (diagnostic): fp32 -> uint8 codes."""
+    _need(x, torch.float32, "x")
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    check(_lib.fp8q_e4m3_encode_f32(x.data_ptr(), x.numel(), out.data_ptr(), _stream(x)), "fp8q_e4m3_encode_f32")
+    return out
+
+
+def device_error(device=None) -> int:
+    """Synchronize the current stream and return (and clear) the device error word."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st, flags = _lib.fp8q_device_error(torch.cuda.current_stream(dev).cuda_stream)
+    if st not in (_lib.FP8Q_OK, _lib.FP8Q_ERR_TIMEOUT, _lib.FP8Q_ERR_DEVICE_CHECK):
+        check(st, "fp8q_device_error")
+    return flags

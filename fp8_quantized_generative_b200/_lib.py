@@ -1,0 +1,113 @@
+"""ctypes binding of libfp8q.so (the C ABI declared in include/fp8q.h).
+
+Argument marshalling only: every entry point here forwards to the function
+of the same name in the shared library.  Pointers are passed as integers
+(device addresses), streams as integers (cudaStream_t handles).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8q.so")
+
+FP8Q_OK = 0
+FP8Q_ERR_INVALID_ARG = 1
+FP8Q_ERR_UNSUPPORTED = 2
+FP8Q_ERR_CUDA = 3
+FP8Q_ERR_TIMEOUT = 4
+FP8Q_ERR_DEVICE_CHECK = 5
+
+DEVERR_TIMEOUT_PRODUCER = 0x1
+DEVERR_TIMEOUT_MMA = 0x2
+DEVERR_TIMEOUT_EPILOGUE = 0x4
+DEVERR_BAD_OFFSETS = 0x8
+DEVERR_TIMEOUT_CLUSTER = 0x10
+
+
+class Fp8qError(RuntimeError):
+    def __init__(self, status: int, what: str, message: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} {message}".rstrip())
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_INT = ctypes.c_int
+
+# name -> (restype, argtypes); mirrors include/fp8q.h
+SIGNATURES = {
+    "fp8q_status_string": (ctypes.c_char_p, [_INT]),
+    "fp8q_last_error_message": (ctypes.c_char_p, []),
+    "fp8q_version": (_INT, []),
+    "fp8q_quantize_rows_dynamic": (_INT, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8q_quantize_weight_per_channel": (_INT, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8q_linear": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "fp8q_moe_grouped_linear": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
+    "fp8q_e4m3_encode_f32": (_INT, [_P, _I64, _P, _P]),
+    "fp8q_device_error": (_INT, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfp8q.so once; fail loudly when it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"fp8q CUDA library missing: {LIB_PATH} — build it with "
+                "`python -m fp8_quantized_generative_b200.build` (there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().fp8q_status_string(int(status)).decode()
+    except ImportError:
+        return f"status {status}"
+
+
+def last_error_message() -> str:
+    return lib().fp8q_last_error_message().decode()
+
+
+def check(status: int, what: str) -> None:
+    if status != FP8Q_OK:
+        raise Fp8qError(status, what, last_error_message())
+
+
+# Raw entry points with the C names (integers in, status out).
+def fp8q_quantize_rows_dynamic(X, M, K, Xq, s_x, stream):
+    return lib().fp8q_quantize_rows_dynamic(X, M, K, Xq, s_x, stream)
+
+
+def fp8q_quantize_weight_per_channel(W, N, K, Wq, s_w, stream):
+    return lib().fp8q_quantize_weight_per_channel(W, N, K, Wq, s_w, stream)
+
+
+def fp8q_linear(Xq, s_x, Wq, s_w, M, N, K, Y, stream):
+    return lib().fp8q_linear(Xq, s_x, Wq, s_w, M, N, K, Y, stream)
+
+
+def fp8q_moe_grouped_linear(Xq, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream):
+    return lib().fp8q_moe_grouped_linear(Xq, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream)
+
+
+def fp8q_e4m3_encode_f32(x, n, out, stream):
+    return lib().fp8q_e4m3_encode_f32(x, n, out, stream)
+
+
+def fp8q_device_error(stream):
+    flags = ctypes.c_uint32(0)
+    st = lib().fp8q_device_error(stream, ctypes.byref(flags))
+    return st, flags.value

@@ -1,0 +1,328 @@
+// FP8 (E4M3 x E4M3) GEMM with FP32 accumulation in tensor memory and a fused
+// per-token x per-channel dequantization + FP16 cast epilogue, for sm_100a.
+//
+// Method: "Quantized Inference for OneRec-V2" (关键证据 steps 3-4: FP8 tensor
+// cores, FP32 accumulation, FP16 output) and
+// "FP8量化在生成式推荐系统OneRec-V2中的优化实践" §2.3 (fused
+// Quantize + GEMM + Dequantize; FP8 multiply + FP32 accumulate + FP16 out)
+// and §3.2 (MoE expert GEMMs, pipelined across experts).
+//
+// One persistent kernel serves both the dense linear and the MoE grouped
+// linear.  Each CTA (one per SM) walks output tiles of 128 x BN:
+//   warp 0      TMA producer: 128-byte-swizzled 2-D tile loads of A (token
+//               rows, K-major) and B (weight rows, K-major) into a STAGES-deep
+//               shared-memory ring, completion tracked by mbarriers;
+//   warp 1      MMA issuer: one thread issues tcgen05.mma kind::f8f6f4
+//               (M=128, N=BN, K=32 per instruction) into one of two TMEM
+//               accumulators, and tcgen05.commit frees smem stages / hands a
+//               finished accumulator to the epilogue;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
+//               output row per thread), y = fp16((acc * s_x[row]) * s_w[col]),
+//               stores masked by the row limit of the tile (the end of the
+//               expert group for MoE) and by N.
+// Two TMEM accumulators let the epilogue of tile i overlap the MMAs of tile
+// i+1.  The MoE tile schedule is built on the device from the expert offsets
+// (no host synchronization): tiles are ordered (expert, n-block, m-block), so
+// the m-blocks that share one expert weight tile run back to back and reuse
+// it from L2.  No TMA multicast is used anywhere.
+#pragma once
+
+#include <cuda.h>
+
+#include "ptx.cuh"
+
+namespace fp8q {
+
+constexpr int kBM = 128;        // rows of an output tile (TMEM lanes)
+constexpr int kBK = 128;        // K bytes per pipeline stage (one 128-B swizzle row)
+constexpr int kUmmaK = 32;      // K per tcgen05.mma for 8-bit operands
+constexpr int kGemmThreads = 192;
+constexpr int kMaxExperts = 4096;
+
+struct GemmParams {
+  const float* s_x;         // [rows]
+  const float* s_w;         // [E*N]
+  __half* Y;                // [rows, N]
+  const int32_t* offsets;   // [E+1] device, grouped only
+  int rows;                 // M (dense) or total grouped rows
+  int N;
+  int K;
+  int E;                    // 1 for dense
+};
+
+template <int BN, int STAGES>
+struct GemmLayout {
+  static constexpr int kABytes = kBM * kBK;
+  static constexpr int kBBytes = BN * kBK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kNumBars = 2 * STAGES + 5;   // full, empty, tfull[2], tempty[2], drain
+  static constexpr int kTmemCols = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+  static constexpr int kFixedBytes = STAGES * kStageBytes + kNumBars * 8 + 32;
+  static size_t smem_bytes(int E) { return 1024 + kFixedBytes + 2 * static_cast<size_t>(E + 1) * 4 + 16; }
+};
+
+struct TileCoord {
+  int a_row0;    // first A (token) row of the tile
+  int row_end;   // rows >= row_end are not stored (end of matrix or of the expert group)
+  int b_row0;    // first B (weight) row
+  int n0;        // first output column
+  int sw0;       // index of s_w for column n0
+};
+
+template <bool kGrouped, int BN>
+__device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p, int num_m, int num_n,
+                                                 const int* tile_prefix, const int* offs) {
+  TileCoord c;
+  if (!kGrouped) {
+    const int m_blk = t % num_m;
+    const int n_blk = t / num_m;
+    c.a_row0 = m_blk * kBM;
+    c.row_end = p.rows;
+    c.n0 = n_blk * BN;
+    c.b_row0 = c.n0;
+    c.sw0 = c.n0;
+  } else {
+    // expert e with tile_prefix[e] <= t < tile_prefix[e+1]
+    int lo = 0, hi = p.E;   // invariant: tile_prefix[lo] <= t < tile_prefix[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tile_prefix[mid] <= t) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int cnt = offs[e + 1] - offs[e];
+    const int mt = (cnt + kBM - 1) / kBM;
+    const int local = t - tile_prefix[e];
+    const int n_blk = local / mt;
+    const int m_loc = local - n_blk * mt;
+    c.a_row0 = offs[e] + m_loc * kBM;
+    c.row_end = offs[e + 1];
+    c.n0 = n_blk * BN;
+    c.b_row0 = e * p.N + c.n0;
+    c.sw0 = e * p.N + c.n0;
+  }
+  return c;
+}
+
+template <int BN, int STAGES, bool kGrouped>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmParams p) {
+  using L = GemmLayout<BN, STAGES>;
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  constexpr uint32_t kIdesc = idesc_e4m3_f32(kBM, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * L::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * L::kBBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* total_s = reinterpret_cast<int*>(tmem_slot + 2);
+  int* tile_prefix = reinterpret_cast<int*>(tmem_slot + 8);
+  int* offs = tile_prefix + (p.E + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_n = (p.N + BN - 1) / BN;
+  const int num_m = (p.rows + kBM - 1) / kBM;
+  const int num_kb = (p.K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4 * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  if (kGrouped) {
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) offs[i] = __ldg(p.offsets + i);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      bool ok = offs[0] == 0 && offs[p.E] == p.rows;
+      int acc = 0;
+      for (int e = 0; e < p.E; ++e) {
+        const int cnt = offs[e + 1] - offs[e];
+        ok = ok && cnt >= 0;
+        tile_prefix[e] = acc;
+        acc += (cnt > 0 ? (cnt + kBM - 1) / kBM : 0) * num_n;
+      }
+      tile_prefix[p.E] = acc;
+      *total_s = ok ? acc : 0;
+      if (!ok && blockIdx.x == 0) raise_error(0x8u);
+    }
+  } else if (threadIdx.x == 0) {
+    *total_s = num_m * num_n;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = *total_s;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, armed = 0, armed_ph = 0;
+      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        const TileCoord c = decode_tile<kGrouped, BN>(t, p, num_m, num_n, tile_prefix, offs);
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+          tma_load_2d(sA + s * L::kABytes, &tmA, &full[s], kb * kBK, c.a_row0);
+          tma_load_2d(sB + s * L::kBBytes, &tmB, &full[s], kb * kBK, c.b_row0);
+          armed |= 1u << s;
+          armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) {
+          raise_error(0x1u);
+          *abort_flag = 1;
+          break;
+        }
+      }
+      // No copy may still be in flight when the CTA exits.
+      for (int i = 0; i < STAGES; ++i)
+        if (armed & (1u << i)) mbar_wait(&full[i], (armed_ph >> i) & 1u, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0, acc = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      bool issued = false;
+      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_ph ^ 1u, abort_flag)) {
+          raise_error(0x2u);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = sw128_kmajor_desc(smem_u32(sA + s * L::kABytes));
+          const uint64_t b0 = sw128_kmajor_desc(smem_u32(sB + s * L::kBBytes));
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k) {
+            // advance the start address by k * 32 bytes inside the swizzle row
+            mma_f8f6f4(d, a0 + static_cast<uint64_t>(k * kUmmaK / 16), b0 + static_cast<uint64_t>(k * kUmmaK / 16),
+                       kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) {
+          raise_error(0x2u);
+          *abort_flag = 1;
+          break;
+        }
+        mma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_ph ^= 1u;
+      }
+      if (issued) {
+        // All issued MMAs must be finished before TMEM is released.
+        mma_commit(drain);
+        mbar_wait(drain, 0, nullptr);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int wq = warp & 3;   // TMEM lane quadrant accessible to this warp
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const TileCoord c = decode_tile<kGrouped, BN>(t, p, num_m, num_n, tile_prefix, offs);
+      if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
+        raise_error(0x4u);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int r = c.a_row0 + wq * 32 + lane;
+      const bool valid = r < c.row_end;
+      const float sx = valid ? __ldg(p.s_x + r) : 0.0f;
+      __half* yrow = p.Y + static_cast<int64_t>(valid ? r : 0) * p.N;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(cc * 32), v);
+        tmem_ld_wait();
+        const int col0 = c.n0 + cc * 32;
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int col = col0 + q * 8;
+            if (col < p.N) {
+              const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.s_w + c.sw0 + cc * 32 + q * 8));
+              const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.s_w + c.sw0 + cc * 32 + q * 8 + 4));
+              const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+              uint32_t packed[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(v[q * 8 + 2 * i]), sx), w[2 * i]);
+                const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(v[q * 8 + 2 * i + 1]), sx), w[2 * i + 1]);
+                const __half2 h = __floats2half2_rn(y0, y1);
+                packed[i] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+              *reinterpret_cast<uint4*>(yrow + col) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_ph ^= 1u;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace fp8q

@@ -1,0 +1,170 @@
+// Per-row dynamic E4M3 quantization (per-token activations at run time,
+// per-output-channel weights offline).  HBM-bound: 2 bytes read and 1 byte
+// written per element plus 4 bytes of scale per row.
+//
+// Method: "Quantized Inference for OneRec-V2" (关键证据, steps 1-2) and
+// "FP8量化在生成式推荐系统OneRec-V2中的优化实践" §2.2 (scale = max_code / max(|x|, eps)),
+// with max_code = 448, the E4M3 maximum (§1.2).
+//
+// Design: a row is held in registers by TPR threads (TPR in {32..256}), each
+// loading VPT 16-byte vectors (8 fp16 values) with coalesced 128-bit loads;
+// the row max is reduced with warp shuffles (plus shared memory across the
+// warps of one row); the codes are then produced from the registers, so X is
+// read from HBM exactly once.  Rows longer than 256 * 8 vectors (K > 16384)
+// fall back to a two-pass loop that re-reads the row (from L2).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fp8q {
+
+constexpr float kE4M3Max = 448.0f;
+constexpr float kScaleEps = 1e-12f;
+
+struct RowScale {
+  float r;  // 448 / a'   (multiplier that maps the row max onto 448)
+  float s;  // a' / 448   (stored dequantization scale)
+};
+
+__device__ __forceinline__ RowScale row_scale_from_amax(float amax) {
+  const float a = fmaxf(amax, kScaleEps);
+  RowScale rs;
+  rs.r = __fdiv_rn(kE4M3Max, a);
+  rs.s = __fdiv_rn(a, kE4M3Max);
+  return rs;
+}
+
+__device__ __forceinline__ float absmax8(const uint4& v, float m) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(h[i]);
+    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+  }
+  return m;
+}
+
+// 8 fp16 -> 8 E4M3 codes (one fp32 multiply by r each, RN), packed little-endian.
+__device__ __forceinline__ uint2 encode8(const uint4& v, float r) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(h[i]);
+    w[i] = cvt_e4m3x2(__fmul_rn(f.x, r), __fmul_rn(f.y, r));
+  }
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// Grid: ceil(M / (256 / TPR)) CTAs of 256 threads; TPR threads per row.
+template <int TPR, int VPT>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const __half* __restrict__ X, int M, int K,
+                                                        uint8_t* __restrict__ Q, float* __restrict__ S) {
+  static_assert(TPR >= 32 && TPR <= 256 && (TPR & (TPR - 1)) == 0, "TPR");
+  constexpr int kRowsPerCta = 256 / TPR;
+  constexpr int kWarpsPerRow = TPR / 32;
+  __shared__ float red[8];
+
+  const int t = threadIdx.x % TPR;
+  const int slot = threadIdx.x / TPR;
+  const int row = blockIdx.x * kRowsPerCta + slot;
+  const bool live = row < M;
+  const int nvec = K >> 3;
+
+  const uint4* src = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(row) * K);
+  uint4 v[VPT];
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int j = t + i * TPR;
+    if (live && j < nvec) {
+      v[i] = __ldg(src + j);
+      m = absmax8(v[i], m);
+    } else {
+      v[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (kWarpsPerRow > 1) {
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) red[warp] = m;
+    __syncthreads();
+    const int w0 = slot * kWarpsPerRow;
+#pragma unroll
+    for (int w = 0; w < kWarpsPerRow; ++w) m = fmaxf(m, red[w0 + w]);
+  }
+  if (!live) return;
+
+  const RowScale rs = row_scale_from_amax(m);
+  uint2* dst = reinterpret_cast<uint2*>(Q + static_cast<int64_t>(row) * K);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int j = t + i * TPR;
+    if (j < nvec) dst[j] = encode8(v[i], rs.r);
+  }
+  if (t == 0) S[row] = rs.s;
+}
+
+// Any K (multiple of 8): one CTA of 256 threads per row, two passes over the row.
+__global__ void __launch_bounds__(256) quant_rows_long_kernel(const __half* __restrict__ X, int M, int K,
+                                                             uint8_t* __restrict__ Q, float* __restrict__ S) {
+  __shared__ float red[8];
+  const int row = blockIdx.x;
+  const int nvec = K >> 3;
+  const uint4* src = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(row) * K);
+  float m = 0.0f;
+  for (int j = threadIdx.x; j < nvec; j += 256) m = absmax8(__ldg(src + j), m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
+  const RowScale rs = row_scale_from_amax(m);
+  uint2* dst = reinterpret_cast<uint2*>(Q + static_cast<int64_t>(row) * K);
+  for (int j = threadIdx.x; j < nvec; j += 256) dst[j] = encode8(__ldg(src + j), rs.r);
+  if (threadIdx.x == 0) S[row] = rs.s;
+}
+
+// Diagnostic elementwise cast (same device cast as the quantizers).
+__global__ void e4m3_encode_kernel(const float* __restrict__ x, int64_t n, uint8_t* __restrict__ out) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; 2 * i < n; i += stride) {
+    const int64_t k = 2 * i;
+    if (k + 1 < n) {
+      const uint16_t c = cvt_e4m3x2(x[k], x[k + 1]);
+      out[k] = static_cast<uint8_t>(c & 0xFF);
+      out[k + 1] = static_cast<uint8_t>(c >> 8);
+    } else {
+      out[k] = static_cast<uint8_t>(cvt_e4m3x2(x[k], 0.0f) & 0xFF);
+    }
+  }
+}
+
+// Host-side launcher: picks (TPR, VPT) so one row fits in registers.
+inline cudaError_t launch_quant_rows(const __half* X, int M, int K, uint8_t* Q, float* S, cudaStream_t st) {
+  const int nvec = K / 8;
+  int tpr = 32;
+  while (tpr < 256 && tpr * 8 < nvec) tpr *= 2;
+  const int vpt_needed = (nvec + tpr - 1) / tpr;
+  if (vpt_needed > 8) {
+    quant_rows_long_kernel<<<M, 256, 0, st>>>(X, M, K, Q, S);
+    return cudaGetLastError();
+  }
+  const int rows_per_cta = 256 / tpr;
+  const dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
+  const int vpt = vpt_needed <= 1 ? 1 : vpt_needed <= 2 ? 2 : vpt_needed <= 4 ? 4 : 8;
+#define FP8Q_QR_CASE(T, V)                                                   \
+  if (tpr == T && vpt == V) {                                                \
+    quant_rows_kernel<T, V><<<grid, 256, 0, st>>>(X, M, K, Q, S);            \
+    return cudaGetLastError();                                               \
+  }
+  FP8Q_QR_CASE(32, 1) FP8Q_QR_CASE(32, 2) FP8Q_QR_CASE(32, 4) FP8Q_QR_CASE(32, 8)
+  FP8Q_QR_CASE(64, 8) FP8Q_QR_CASE(128, 8) FP8Q_QR_CASE(256, 8)
+  FP8Q_QR_CASE(64, 4) FP8Q_QR_CASE(128, 4) FP8Q_QR_CASE(256, 4)
+#undef FP8Q_QR_CASE
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace fp8q

@@ -1,0 +1,153 @@
+/*
+ * fp8q — FP8 W8A8 linear layers for NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * The method (two web pages on quantized inference for the OneRec-V2
+ * generative recommender):
+ *   [P1] "Quantized Inference for OneRec-V2：生成式推荐开始直接吃 LLM 量化栈",
+ *        section 关键证据: linear weights quantized offline per output
+ *        channel; activations quantized per token at run time; the matmul runs
+ *        on FP8 tensor cores with FP32 accumulation; the output is cast back to
+ *        FP16.  Covered layers: attention QKV/O projections, dense FFN linears
+ *        and the sparse-MoE expert grouped GEMM.
+ *   [P2] "FP8量化在生成式推荐系统OneRec-V2中的优化实践", §1.2 (FP8 range ±448),
+ *        §2.2 (E4M3; per-token dynamic scale = max_code / max(|x|, eps)),
+ *        §2.3 (FP8 multiply + FP32 accumulate + FP16 output, Q+GEMM+DQ fused).
+ *
+ * Numerics, identical in every entry point:
+ *   per row:  a' = max(max_k |A[k]|, 1e-12f)
+ *             r  = 448 / a'   (IEEE fp32 division, round to nearest)
+ *             s  = a' / 448   (IEEE fp32 division, round to nearest; stored)
+ *             q[k] = E4M3(fl32(A[k] * r)), round-to-nearest-even, saturating
+ *                    to ±448; -0.0 keeps its sign.
+ *   linear:   Y[m,n] = fp16_rn( fl32( fl32(acc[m,n] * s_x[m]) * s_w[n] ) ),
+ *             acc = FP32 tensor-core accumulation of E4M3 x E4M3 products.
+ *
+ * Conventions for every entry point:
+ *   - Matrices are row-major and dense.  X, W and Y are fp16 ([M,K], [N,K],
+ *     [M,N]; K is the contiguous dimension of X and W, like nn.Linear);
+ *     E4M3 codes are uint8 with the same layout as their source.
+ *   - Every pointer argument is a CUDA device pointer owned by the caller,
+ *     allocated on the device that is current when the call is made, and
+ *     16-byte aligned.  Outputs must not alias inputs.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work and return; they never synchronize, except
+ *     fp8q_device_error().
+ *   - Arguments are validated on the host before anything is enqueued; a
+ *     rejected call enqueues nothing and returns FP8Q_ERR_INVALID_ARG or
+ *     FP8Q_ERR_UNSUPPORTED.  A failed launch returns FP8Q_ERR_CUDA
+ *     (fp8q_last_error_message() holds the CUDA error text).
+ *   - Shape rules: M, rows >= 0 (0 is a no-op), N > 0, K > 0, K % 16 == 0
+ *     (16-byte TMA rows for the FP8 operands), N % 8 == 0 (16-byte fp16
+ *     output rows), all sizes < 2^31.
+ *   - Kernels bound every wait on the GPU (about 2 s); a wait that runs out
+ *     sets a device error word instead of hanging, readable with
+ *     fp8q_device_error().
+ *   - No call allocates device memory.  Results are bitwise reproducible from
+ *     run to run (fixed reduction order everywhere).
+ */
+#ifndef FP8Q_H_
+#define FP8Q_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP8Q_OK = 0,
+  FP8Q_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment       */
+  FP8Q_ERR_UNSUPPORTED = 2,   /* valid request this build cannot serve      */
+  FP8Q_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed          */
+  FP8Q_ERR_TIMEOUT = 4,       /* a device wait ran out (fp8q_device_error)  */
+  FP8Q_ERR_DEVICE_CHECK = 5   /* a device-side input check failed           */
+} fp8q_status;
+
+/* Device error-word bits reported by fp8q_device_error(). */
+#define FP8Q_DEVERR_TIMEOUT_PRODUCER 0x1u
+#define FP8Q_DEVERR_TIMEOUT_MMA      0x2u
+#define FP8Q_DEVERR_TIMEOUT_EPILOGUE 0x4u
+#define FP8Q_DEVERR_BAD_OFFSETS      0x8u
+#define FP8Q_DEVERR_TIMEOUT_CLUSTER  0x10u
+
+/* Human-readable name of a status code.  Never returns NULL. */
+const char* fp8q_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* fp8q_last_error_message(void);
+
+/* ABI version of this library (major * 100 + minor). */
+int fp8q_version(void);
+
+/*
+ * Per-token dynamic activation quantization  [P1 关键证据 step 2; P2 §2.2].
+ *   X_f16 [M,K] fp16 in;  Xq [M,K] uint8 E4M3 out;  s_x [M] fp32 out.
+ * One scale per row, computed at run time from the row's max |x|.
+ * M == 0 is a no-op.
+ */
+fp8q_status fp8q_quantize_rows_dynamic(const void* X_f16, int64_t M, int64_t K,
+                                       uint8_t* Xq, float* s_x, void* stream);
+
+/*
+ * Per-output-channel weight quantization, done once offline  [P1 关键证据
+ * step 1; P2 §2.1 per-channel for the QKV projection].
+ *   W_f16 [N,K] fp16 in;  Wq [N,K] uint8 E4M3 out;  s_w [N] fp32 out.
+ * For MoE expert weights [E,N_e,K] pass N = E * N_e (one scale per row of
+ * every expert).  Same arithmetic as fp8q_quantize_rows_dynamic.
+ */
+fp8q_status fp8q_quantize_weight_per_channel(const void* W_f16, int64_t N, int64_t K,
+                                             uint8_t* Wq, float* s_w, void* stream);
+
+/*
+ * FP8 W8A8 linear with fused dequantization  [P1 关键证据 steps 3-4;
+ * P2 §2.3 "FP8 multiply + FP32 accumulate + FP16 output"].
+ *   Xq [M,K] uint8, s_x [M] fp32, Wq [N,K] uint8, s_w [N] fp32 in;
+ *   Y_f16 [M,N] fp16 out:  Y = fp16(((Xq . Wq^T) * s_x[:,None]) * s_w[None,:]).
+ * M == 0 is a no-op.
+ */
+fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x,
+                        const uint8_t* Wq, const float* s_w,
+                        int64_t M, int64_t N, int64_t K,
+                        void* Y_f16, void* stream);
+
+/*
+ * MoE expert grouped FP8 linear  [P1 关键证据 item 2: Sparse MoE grouped
+ * GEMM; P2 §3.2 MoE acceleration].
+ *   Xq [rows,K] uint8 and s_x [rows] fp32: token rows already grouped by
+ *       expert (rows offsets[e] .. offsets[e+1]-1 go to expert e);
+ *   offsets [E+1] int32, DEVICE memory, non-decreasing, offsets[0] == 0,
+ *       offsets[E] == rows (read on the device; the host never syncs on it);
+ *   Wq [E,N,K] uint8 and s_w [E,N] fp32: per-expert weights and
+ *       per-channel scales;
+ *   Y_f16 [rows,N] fp16 out: row i of group e = linear of that row with W_e.
+ * Empty groups are legal.  Offsets that break the rules are detected on the
+ * device: nothing is written and fp8q_device_error() reports
+ * FP8Q_DEVERR_BAD_OFFSETS.  E >= 1 and E <= 4096.
+ */
+fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x,
+                                    const int32_t* offsets, int32_t E, int64_t rows,
+                                    const uint8_t* Wq, const float* s_w,
+                                    int64_t N, int64_t K,
+                                    void* Y_f16, void* stream);
+
+/*
+ * Diagnostic: the device E4M3 cast on its own, out[i] = E4M3(x[i]) with the
+ * same rounding as the quantizers (RNE, saturating to ±448).  n >= 0,
+ * x and out need no particular alignment.  Exists so that the cast can be
+ * checked against an independent encoder over arbitrary fp32 bit patterns.
+ */
+fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device error word of the
+ * current device (an OR of FP8Q_DEVERR_* bits, 0 if none).  Returns
+ * FP8Q_ERR_TIMEOUT if a timeout bit was set, FP8Q_ERR_DEVICE_CHECK if only
+ * input-check bits were set, FP8Q_OK otherwise.  `flags` may be NULL.
+ */
+fp8q_status fp8q_device_error(void* stream, uint32_t* flags);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* FP8Q_H_ */

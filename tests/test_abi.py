@@ -1,0 +1,102 @@
+"""The C ABI library loads, exports every symbol declared in include/fp8q.h,
+and rejects bad arguments on the host before touching the GPU (no GPU needed)."""
+import os
+import re
+
+import pytest
+
+from fp8_quantized_generative_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8q.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8q_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(_lib.LIB_PATH):
+        from fp8_quantized_generative_b200 import build
+        build.build()
+    return _lib.lib()
+
+
+def test_header_declares_the_path_entry_points():
+    names = declared_functions()
+    for required in ("fp8q_quantize_weight_per_channel", "fp8q_quantize_rows_dynamic", "fp8q_linear",
+                     "fp8q_moe_grouped_linear"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings(L):
+    assert _lib.status_string(0) == "FP8Q_OK"
+    assert _lib.status_string(1) == "FP8Q_ERR_INVALID_ARG"
+    assert _lib.status_string(99) == "FP8Q_UNKNOWN_STATUS"
+    assert L.fp8q_version() >= 100
+
+
+BAD = 0x1008   # 8-byte aligned, not 16
+
+
+@pytest.mark.parametrize("args", [
+    (0, 4, 32, 0x1000, 0x2000, 0),          # null X
+    (0x1000, 4, 32, 0, 0x2000, 0),          # null Xq
+    (0x1000, -1, 32, 0x1000, 0x2000, 0),    # negative M
+    (0x1000, 4, 0, 0x1000, 0x2000, 0),      # K = 0
+    (0x1000, 4, 24, 0x1000, 0x2000, 0),     # K % 16 != 0
+    (BAD, 4, 32, 0x1000, 0x2000, 0),        # misaligned
+])
+def test_quantize_rejects(L, args):
+    assert _lib.fp8q_quantize_rows_dynamic(*args) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.last_error_message() != ""
+
+
+def test_quantize_zero_rows_is_noop(L):
+    assert _lib.fp8q_quantize_rows_dynamic(0, 0, 32, 0, 0, 0) == _lib.FP8Q_OK
+    assert _lib.fp8q_quantize_weight_per_channel(0, 0, 32, 0, 0, 0) == _lib.FP8Q_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("M,N,K,ptrs", [
+    (4, 0, 32, None), (4, 12, 32, None), (4, 16, 40, None), (-2, 16, 32, None),
+    (4, 16, 32, (0, 0x1000, 0x1000, 0x1000, 0x1000)),
+    (4, 16, 32, (0x1000, 0x1000, BAD, 0x1000, 0x1000)),
+])
+def test_linear_rejects(L, M, N, K, ptrs):
+    p = ptrs or (0x1000,) * 5
+    assert _lib.fp8q_linear(p[0], p[1], p[2], p[3], M, N, K, p[4], 0) == _lib.FP8Q_ERR_INVALID_ARG
+
+
+def test_linear_zero_rows_is_noop(L):
+    assert _lib.fp8q_linear(0, 0, 0, 0, 0, 16, 32, 0, 0) == _lib.FP8Q_OK
+
+
+@pytest.mark.parametrize("E,rows,N,K,off", [
+    (0, 8, 16, 32, 0x1000), (4097, 8, 16, 32, 0x1000), (4, 8, 12, 32, 0x1000),
+    (4, 8, 16, 20, 0x1000), (4, 8, 16, 32, 0), (4, 8, 16, 32, 0x1002), (4, -1, 16, 32, 0x1000),
+])
+def test_moe_rejects(L, E, rows, N, K, off):
+    a = 0x1000
+    assert _lib.fp8q_moe_grouped_linear(a, a, off, E, rows, a, a, N, K, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+
+
+def test_encode_rejects(L):
+    assert _lib.fp8q_e4m3_encode_f32(0, 10, 0x1000, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_e4m3_encode_f32(0x1000, -1, 0x1000, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_e4m3_encode_f32(0, 0, 0, 0) == _lib.FP8Q_OK
+
+
+def test_python_wrappers_refuse_cpu_tensors():
+    import torch
+    import fp8_quantized_generative_b200 as fq
+    with pytest.raises(ValueError):
+        fq.quantize_rows_dynamic(torch.zeros(4, 32, dtype=torch.float16))

@@ -1,0 +1,109 @@
+"""GPU parity of the FP8 W8A8 linear (quantize + tcgen05 GEMM + fused dequant).
+
+Each case draws seeded fp16 X and W, runs the library path (per-token
+quantization, per-channel weight quantization, fp8q_linear) and compares the
+fp16 output with the CPU oracle (quant_rows + linear_ref in float64) computed
+from the same fp16 inputs.  Full-size workloads are compared on sampled rows
+(the oracle is row-separable, so a sampled row is checked exactly as in the
+full problem); small and ragged shapes are compared element by element.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import linear_ref, quant_rows
+from fp8_quantized_generative_b200 import workloads as wl
+
+from parity import assert_close_f16, assert_no_device_error, sample_rows, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fq():
+    import fp8_quantized_generative_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def run_gpu(fq, X, W):
+    Xd, Wd = X.cuda(), W.cuda()
+    Wq, s_w = fq.quantize_weight_per_channel(Wd)
+    Xq, s_x = fq.quantize_rows_dynamic(Xd)
+    Y = fq.linear(Xq, s_x, Wq, s_w)
+    torch.cuda.synchronize()
+    return Y
+
+
+def oracle_rows(X, W, rows):
+    Wq, s_w = quant_rows(W.numpy())
+    Xq, s_x = quant_rows(X.numpy()[rows])
+    return linear_ref(Xq, s_x, Wq, s_w)
+
+
+def check(fq, X, W, n_rows=None, what=""):
+    Y = run_gpu(fq, X, W)
+    rows = np.arange(X.shape[0]) if n_rows is None else sample_rows(X.shape[0], n_rows, seed=X.shape[0])
+    assert_close_f16(to_np(Y)[rows], oracle_rows(X, W, rows), what)
+    assert_no_device_error()
+    return Y
+
+
+def test_tiny(fq):
+    lin = wl.tiny()
+    check(fq, lin.X, lin.W, what="tiny")
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 256, 128), (128, 256, 128), (300, 520, 272), (257, 264, 1040), (77, 1000, 16), (1000, 8, 64),
+    (640, 768, 4096),
+])
+def test_ragged_and_multi_tile(fq, M, N, K):
+    X = wl.random_f16((M, K), seed=M + N + K)
+    W = wl.random_f16((N, K), seed=M * N + K, std=0.02)
+    check(fq, X, W, what=f"{M}x{N}x{K}")
+
+
+def test_edge_values(fq):
+    K, N = 256, 256
+    X = wl.random_f16((8, K), seed=3).float()
+    X[0] = 0.0                  # zero row -> zero output row
+    X[1, 5] = 65504.0           # huge outlier
+    X[2] = 448.0
+    W = wl.random_f16((N, K), seed=4, std=0.02).float()
+    W[7] = 0.0                  # zero channel
+    Y = check(fq, X.half(), W.half(), what="edge")
+    y = to_np(Y).astype(np.float64)
+    assert np.all(y[0] == 0) and np.all(y[:, 7] == 0)
+
+
+def test_qkv_full(fq):
+    lin = wl.qkv()
+    check(fq, lin.X, lin.W, n_rows=192, what="qkv 4096x6144x2048")
+
+
+def test_ffn_full(fq):
+    up, down = wl.ffn()
+    check(fq, up.X, up.W, n_rows=128, what="ffn up 8192x8192x2048")
+    check(fq, down.X, down.W, n_rows=96, what="ffn down 8192x2048x8192")
+
+
+@pytest.mark.parametrize("m", wl.SWEEP_M)
+def test_sweep(fq, m):
+    check(fq, wl.sweep_x(m), wl.sweep_w(), n_rows=min(m, 128), what=f"sweep m={m}")
+
+
+def test_deterministic(fq):
+    lin = wl.qkv(m=512)
+    a = run_gpu(fq, lin.X, lin.W)
+    b = run_gpu(fq, lin.X, lin.W)
+    assert torch.equal(a, b)
+
+
+def test_zero_rows_noop(fq):
+    Xq = torch.empty((0, 128), dtype=torch.uint8, device="cuda")
+    s = torch.empty((0,), dtype=torch.float32, device="cuda")
+    Wq = torch.zeros((64, 128), dtype=torch.uint8, device="cuda")
+    sw = torch.ones((64,), dtype=torch.float32, device="cuda")
+    Y = fq.linear(Xq, s, Wq, sw)
+    assert Y.shape == (0, 64)

@@ -1,0 +1,116 @@
+"""GPU parity of the MoE expert grouped FP8 linear (fp8q_moe_grouped_linear).
+
+Rows arrive grouped by expert (FP16 top-2 router and permutation are part of
+the seeded input synthesis); offsets live on the device.  The oracle computes
+every checked row with its expert's quantized weights and scales.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import linear_ref, moe_ref, quant_rows
+from fp8_quantized_generative_b200 import workloads as wl
+
+from parity import assert_close_f16, assert_no_device_error, sample_rows, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fq():
+    import fp8_quantized_generative_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def run_gpu(fq, Xg, offsets, W):
+    Wq, s_w = fq.quantize_weight_per_channel(W.cuda())
+    Xq, s_x = fq.quantize_rows_dynamic(Xg.cuda())
+    off = torch.from_numpy(np.asarray(offsets, dtype=np.int32)).cuda()
+    Y = fq.moe_grouped_linear(Xq, s_x, off, Wq, s_w)
+    torch.cuda.synchronize()
+    return Y
+
+
+def oracle_rows(Xg, offsets, W, rows):
+    """Oracle output for the given rows only: each row with its own expert."""
+    offsets = np.asarray(offsets, dtype=np.int64)
+    E, N, K = W.shape
+    expert_of = np.searchsorted(offsets, rows, side="right") - 1
+    out = np.zeros((len(rows), N), np.float16)
+    Xq, s_x = quant_rows(Xg.numpy()[rows])
+    for e in np.unique(expert_of):
+        sel = expert_of == e
+        Wq, s_w = quant_rows(W[e].numpy())
+        out[sel] = linear_ref(Xq[sel], s_x[sel], Wq, s_w)
+    return out
+
+
+def test_small_groups_full_compare(fq):
+    E, N, K = 6, 264, 272
+    counts = [0, 130, 1, 0, 300, 57]
+    off = wl.offsets_from_counts(counts)
+    R = int(off[-1])
+    X = wl.random_f16((R, K), seed=11)
+    W = wl.random_f16((E, N, K), seed=12, std=0.02)
+    Y = run_gpu(fq, X, off, W)
+    Wq, s_w = quant_rows(W.reshape(E * N, K).numpy())
+    Xq, s_x = quant_rows(X.numpy())
+    ref = moe_ref(Xq, s_x, off, Wq.reshape(E, N, K), s_w.reshape(E, N))
+    assert_close_f16(to_np(Y), ref, "small groups")
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("counts", [
+    [0, 0, 0, 513, 0],            # one expert holds every row
+    [1, 1, 1, 1, 1, 1, 1, 1],     # single-row groups
+    [128, 128, 256],              # exact tile multiples
+    [700],                        # E = 1 behaves like a dense linear
+])
+def test_adversarial_offsets(fq, counts):
+    E, N, K = len(counts), 256, 256
+    off = wl.offsets_from_counts(counts)
+    R = int(off[-1])
+    X = wl.random_f16((R, K), seed=R + E)
+    W = wl.random_f16((E, N, K), seed=E + 1, std=0.02)
+    Y = run_gpu(fq, X, off, W)
+    assert_close_f16(to_np(Y), oracle_rows(X, off, W, np.arange(R)), f"counts={counts}")
+    assert_no_device_error()
+
+
+def test_bad_offsets_are_reported_and_nothing_written(fq):
+    E, N, K = 3, 64, 128
+    X = wl.random_f16((10, K), seed=1).cuda()
+    Xq, s_x = fq.quantize_rows_dynamic(X)
+    Wq = torch.zeros((E, N, K), dtype=torch.uint8, device="cuda")
+    s_w = torch.ones((E, N), dtype=torch.float32, device="cuda")
+    for bad in ([0, 6, 4, 10], [1, 4, 6, 10], [0, 4, 6, 9]):
+        off = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        Y = torch.full((10, N), 7.0, dtype=torch.float16, device="cuda")
+        fq.moe_grouped_linear(Xq, s_x, off, Wq, s_w, out=Y)
+        flags = fq.device_error()
+        assert flags == 0x8, hex(flags)
+        assert torch.all(Y == 7.0)
+
+
+@pytest.fixture(scope="module")
+def moe_case():
+    return wl.moe()
+
+
+def test_moe_up_full(fq, moe_case):
+    m = moe_case
+    Y = run_gpu(fq, m.X_perm, m.offsets, m.W_up)
+    rows = sample_rows(m.X_perm.shape[0], 256, seed=4)
+    assert_close_f16(to_np(Y)[rows], oracle_rows(m.X_perm, m.offsets, m.W_up, rows), "moe up")
+    assert_no_device_error()
+
+
+def test_moe_down_full(fq, moe_case):
+    # Down projection on an independent seeded input of the up-output's shape.
+    m = moe_case
+    Xd = wl.random_f16((m.X_perm.shape[0], wl.MOE_F), seed=303)
+    Y = run_gpu(fq, Xd, m.offsets, m.W_down)
+    rows = sample_rows(Xd.shape[0], 256, seed=5)
+    assert_close_f16(to_np(Y)[rows], oracle_rows(Xd, m.offsets, m.W_down, rows), "moe down")
+    assert_no_device_error()

@@ -414,6 +414,8 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(device)
     barrier = make_barrier(world, device)
     desc, kind, tensors = workload_spec(args.workload)
+    import fp8_quantized_generative_b200 as fq
+    fq.set_gemm_tuning({"auto": 0, "single": 1, "pair": 2}[args.gemm], args.bn)
     plan = Plan(kind, tensors, device, min_rotation_bytes=3 * L2_BYTES)
     peaks, peak_src = load_peaks()
 
@@ -469,6 +471,7 @@ def run_ours(args, world, rank, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3 (fp32 accumulate, fp16 out)",
             "data": "synthetic",
             "config": {"workload": desc, "parallelism": f"replicas x{world} (no collective)",
+                       "gemm": args.gemm, "bn": args.bn,
                        "l2": f"rotating {plan.sets} buffer sets of {plan.bytes_per_set / 1e6:.0f} MB "
                              f"(> 3x 126 MB L2), no flush",
                        "step": " -> ".join(plan.kernels)},
@@ -502,6 +505,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="qkv")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm", default="auto", choices=["auto", "single", "pair"],
+                    help="dense GEMM kernel family (tuning sweeps; default: chosen per shape)")
+    ap.add_argument("--bn", type=int, default=0, help="pair-kernel tile width (0 = automatic)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -21,7 +21,7 @@ from ._lib import Fp8qError, check, lib
 
 __all__ = [
     "Fp8qError", "lib", "quantize_rows_dynamic", "quantize_weight_per_channel", "linear",
-    "moe_grouped_linear", "quantized_linear", "e4m3_encode_f32", "device_error",
+    "moe_grouped_linear", "quantized_linear", "e4m3_encode_f32", "device_error", "set_gemm_tuning",
 ]
 
 
@@ -116,6 +116,11 @@ def e4m3_encode_f32(x: torch.Tensor) -> torch.Tensor:
     out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     check(_lib.fp8q_e4m3_encode_f32(x.data_ptr(), x.numel(), out.data_ptr(), _stream(x)), "fp8q_e4m3_encode_f32")
     return out
+
+
+def set_gemm_tuning(kernel_family: int = 0, tile_n: int = 0) -> None:
+    """Override the dense-linear kernel choice (0 = automatic; see include/fp8q.h)."""
+    check(_lib.fp8q_set_gemm_tuning(kernel_family, tile_n), "fp8q_set_gemm_tuning")
 
 
 def device_error(device=None) -> int:

@@ -6,12 +6,15 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <climits>
 #include <mutex>
 #include <string>
 
 #include "fp8q.h"
 #include "gemm_fp8.cuh"
+#include "gemm_fp8_pair.cuh"
 #include "quant_rows.cuh"
 
 namespace fp8q {
@@ -98,9 +101,81 @@ fp8q_status make_operand_map(CUtensorMap* m, const void* base, int64_t rows, int
   return FP8Q_OK;
 }
 
+// fp16 output [rows, N] written in 32 x 32 boxes through a 64-byte-swizzled
+// staging tile; the store clips rows >= rows and columns >= N.
+fp8q_status make_output_map(CUtensorMap* m, const void* base, int64_t rows, int64_t N) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) {
+    g_last_error = "cuTensorMapEncodeTiled entry point unavailable";
+    return FP8Q_ERR_CUDA;
+  }
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[96];
+    std::snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled(output) failed (CUresult %d)", static_cast<int>(r));
+    g_last_error = buf;
+    return FP8Q_ERR_CUDA;
+  }
+  return FP8Q_OK;
+}
+
 // ------------------------------------------------------------------ GEMM launch
 constexpr int kBN = 256;
 constexpr int kStages = 4;
+
+// Tuning knobs read once from the environment (for measurement sweeps):
+//   FP8Q_FORCE_KERNEL = auto | single | pair   (dense linear kernel family)
+//   FP8Q_BN           = 0 (auto) | 128 | 192 | 256   (pair-kernel tile width)
+// fp8q_set_gemm_tuning() overrides both at run time.
+struct Knobs {
+  int force = 0;  // 0 auto, 1 single, 2 pair
+  int bn = 0;
+};
+Knobs& knobs() {
+  static Knobs k = []() {
+    Knobs r;
+    if (const char* f = std::getenv("FP8Q_FORCE_KERNEL")) {
+      if (!std::strcmp(f, "single")) r.force = 1;
+      if (!std::strcmp(f, "pair")) r.force = 2;
+    }
+    if (const char* b = std::getenv("FP8Q_BN")) r.bn = std::atoi(b);
+    return r;
+  }();
+  return k;
+}
+
+template <typename... Args>
+cudaError_t launch_ex(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
+                      bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 template <bool kGrouped>
 fp8q_status launch_gemm(const uint8_t* A, int64_t a_rows, const uint8_t* B, int64_t b_rows, const GemmParams& p,
@@ -114,15 +189,124 @@ fp8q_status launch_gemm(const uint8_t* A, int64_t a_rows, const uint8_t* B, int6
   if (s != FP8Q_OK) return s;
   s = make_operand_map(&tb, B, b_rows, p.K, kBN);
   if (s != FP8Q_OK) return s;
+  CUtensorMap ty;
+  s = make_output_map(&ty, p.Y, p.rows, p.N);
+  if (s != FP8Q_OK) return s;
   auto kernel = fp8_gemm_kernel<kBN, kStages, kGrouped>;
   const size_t smem = L::smem_bytes(kGrouped ? p.E : 0);
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   const int grid = static_cast<int>(tiles_upper_bound < sms ? (tiles_upper_bound < 1 ? 1 : tiles_upper_bound) : sms);
-  kernel<<<grid, kGemmThreads, smem, st>>>(ta, tb, p);
-  e = cudaGetLastError();
+  e = launch_ex(kernel, dim3(grid), dim3(kGemmThreads), smem, st, 1, true, ta, tb, ty, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_kernel launch");
   return FP8Q_OK;
+}
+
+// Per-device cache of how many 2-CTA clusters of a pair kernel fit at once.
+template <int BN, int STAGES>
+int max_pair_clusters(int dev) {
+  static int cache[kMaxDevices] = {0};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  if (cache[dev] > 0) return cache[dev];
+  using L = PairLayout<BN, STAGES>;
+  auto kernel = fp8_gemm_pair_kernel<BN, STAGES>;
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L::kSmemBytes));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = L::kSmemBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  cache[dev] = n;
+  return n;
+}
+
+template <int BN, int STAGES>
+fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, const GemmParams& p, int dev, cudaStream_t st) {
+  using L = PairLayout<BN, STAGES>;
+  CUtensorMap ta, tb;
+  fp8q_status s = make_operand_map(&ta, A, p.rows, p.K, kBM);
+  if (s != FP8Q_OK) return s;
+  s = make_operand_map(&tb, B, p.N, p.K, L::kBRows);
+  if (s != FP8Q_OK) return s;
+  CUtensorMap ty;
+  s = make_output_map(&ty, p.Y, p.rows, p.N);
+  if (s != FP8Q_OK) return s;
+  auto kernel = fp8_gemm_pair_kernel<BN, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::kSmemBytes));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair)");
+  const int clusters = max_pair_clusters<BN, STAGES>(dev);
+  if (clusters < 1) {
+    g_last_error = "no 2-CTA cluster of the pair GEMM fits on this device";
+    return FP8Q_ERR_UNSUPPORTED;
+  }
+  const int64_t tiles = int64_t((p.rows + 2 * kBM - 1) / (2 * kBM)) * ((p.N + BN - 1) / BN);
+  const int pairs = static_cast<int>(tiles < clusters ? tiles : clusters);
+  e = launch_ex(kernel, dim3(2 * pairs), dim3(kGemmThreads), L::kSmemBytes, st, 2, true, ta, tb, ty, p);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_pair_kernel launch");
+  return FP8Q_OK;
+}
+
+// Pair-kernel tile width: the candidate with the least modelled time =
+// waves of tiles x per-tile work / relative efficiency.  Narrower tiles move
+// more operand bytes out of L2 per FLOP (256 FLOP/B per SM at BN = 256,
+// 219 at 192, 171 at 128) and pay the per-tile epilogue more often; the
+// efficiency factors are per-FLOP throughputs relative to BN = 256 measured
+// on B200 (4096 x 6144 x 2048).  A narrower tile only wins when it removes a
+// mostly idle wave.
+int choose_pair_bn(int64_t M, int64_t N, int clusters) {
+  const int cands[3] = {256, 192, 128};
+  const double eff[3] = {1.0, 0.79, 0.60};
+  int best = 256;
+  double best_cost = 1e300;
+  for (int i = 0; i < 3; ++i) {
+    const int bn = cands[i];
+    const int64_t tiles = ((M + 255) / 256) * ((N + bn - 1) / bn);
+    const int64_t waves = (tiles + clusters - 1) / clusters;
+    const double cost = static_cast<double>(waves) * bn / eff[i];
+    if (cost < best_cost * 0.999) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams& p, cudaStream_t st) {
+  int dev = 0, sms = 0;
+  cudaError_t e = current_device_info(&dev, &sms);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  const Knobs kn = knobs();
+  bool pair = p.rows > kBM;
+  // Walk n-blocks first when A is the larger operand: each A block is then
+  // reused by every n-block while it is in L2, and the smaller B stays there.
+  GemmParams q = p;
+  q.n_fastest = int64_t(p.rows) > int64_t(p.N) ? 1 : 0;
+  if (kn.force == 1) pair = false;
+  if (kn.force == 2) pair = true;
+  if (pair) {
+    const int clusters = max_pair_clusters<256, 6>(dev);
+    int bn = kn.bn ? kn.bn : choose_pair_bn(p.rows, p.N, clusters > 0 ? clusters : sms / 2);
+    switch (bn) {
+      case 128: return launch_pair<128, 8>(Xq, Wq, q, dev, st);
+      case 192: return launch_pair<192, 7>(Xq, Wq, q, dev, st);
+      default: return launch_pair<256, 6>(Xq, Wq, q, dev, st);
+    }
+  }
+  const int64_t tiles = int64_t((p.rows + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
+  return launch_gemm<false>(Xq, p.rows, Wq, p.N, q, tiles, st);
 }
 
 fp8q_status check_quant_args(const void* X, int64_t M, int64_t K, const void* Q, const void* S) {
@@ -195,14 +379,14 @@ fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, 
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.E = 1;
-  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
-  return launch_gemm<false>(Xq, M, Wq, N, p, tiles, static_cast<cudaStream_t>(stream));
+  p.n_fastest = 0;
+  return launch_dense(Xq, Wq, p, static_cast<cudaStream_t>(stream));
 }
 
 fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const int32_t* offsets, int32_t E,
                                     int64_t rows, const uint8_t* Wq, const float* s_w, int64_t N, int64_t K,
                                     void* Y_f16, void* stream) {
-  if (E < 1 || E > kMaxExperts) return invalid("E must be in [1, 4096]");
+  if (E < 1 || E > kMaxExperts) return invalid("E must be in [1, 1024]");
   if (rows < 0 || rows > kMaxDim) return invalid("rows out of range");
   if (N <= 0 || N % 8 != 0 || int64_t(E) * N > kMaxDim) return invalid("N must be positive, a multiple of 8, E*N < 2^31");
   if (K <= 0 || K > kMaxDim || K % 16 != 0) return invalid("K must be positive and a multiple of 16");
@@ -219,6 +403,7 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const i
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.E = E;
+  p.n_fastest = 0;
   const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBN - 1) / kBN);
   return launch_gemm<true>(Xq, rows, Wq, int64_t(E) * N, p, tiles, static_cast<cudaStream_t>(stream));
 }
@@ -236,6 +421,14 @@ fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* 
   e4m3_encode_kernel<<<static_cast<int>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, n, out);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "e4m3_encode launch");
+  return FP8Q_OK;
+}
+
+fp8q_status fp8q_set_gemm_tuning(int kernel_family, int tile_n) {
+  if (kernel_family < 0 || kernel_family > 2) return invalid("kernel_family must be 0, 1 or 2");
+  if (tile_n != 0 && tile_n != 128 && tile_n != 192 && tile_n != 256) return invalid("tile_n must be 0, 128, 192 or 256");
+  knobs().force = kernel_family;
+  knobs().bn = tile_n;
   return FP8Q_OK;
 }
 

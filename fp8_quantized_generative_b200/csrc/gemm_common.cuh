@@ -1,0 +1,120 @@
+// Pieces shared by the single-CTA and CTA-pair FP8 GEMM kernels: problem
+// parameters, warp roles and the fused dequantization epilogue.
+//
+// Epilogue arithmetic ("Quantized Inference for OneRec-V2", 关键证据 steps
+// 3-4; "FP8量化在生成式推荐系统OneRec-V2中的优化实践" §2.3): the FP32
+// accumulator of output (m, n) is scaled by the per-token scale s_x[m] and the
+// per-channel scale s_w[n], in that order, each an fp32 multiply rounded to
+// nearest, and cast once to fp16 (round to nearest even).
+#pragma once
+
+#include <cuda.h>
+
+#include "ptx.cuh"
+
+namespace fp8q {
+
+constexpr int kBM = 128;          // rows of a CTA's output slab (TMEM lanes)
+constexpr int kBK = 128;          // K bytes per pipeline stage (one 128-B swizzle row)
+constexpr int kUmmaK = 32;        // K per tcgen05.mma for 8-bit operands
+constexpr int kEpiWarp0 = 2;      // warps 0, 1: TMA producer, MMA issuer
+constexpr int kEpiWarps = 8;      // two epilogue warps per TMEM lane quadrant
+constexpr int kGemmThreads = (kEpiWarp0 + kEpiWarps) * 32;
+constexpr int kStageTileBytes = 32 * 32 * 2;   // one 32 x 32 fp16 output tile per epilogue warp
+constexpr int kEpiSmemBytes = kEpiWarps * kStageTileBytes;
+constexpr int kMaxExperts = 1024;
+
+struct GemmParams {
+  const float* s_x;         // [rows]
+  const float* s_w;         // [E*N]
+  __half* Y;                // [rows, N]
+  const int32_t* offsets;   // [E+1] device, grouped only
+  int rows;                 // M (dense) or total grouped rows
+  int N;
+  int K;
+  int E;                    // 1 for dense
+  int n_fastest;            // dense tile order: 1 = walk n-blocks first
+};
+
+// One output slab of a CTA: 128 rows starting at row0, BN columns at n0.
+struct EpiTile {
+  int row0;
+  int row_end;   // rows >= row_end are not stored
+  int n0;
+  int sw0;       // index into s_w of column n0
+  bool tma;      // the bulk tensor store may write the whole slab
+};
+
+// Staging layout of a 32 x 32 fp16 tile: row r occupies 64 bytes, its four
+// 16-byte chunks permuted as chunk c -> c ^ ((r >> 1) & 3).  This is the
+// layout a 64-byte-swizzled TMA box of 32 x 32 fp16 expects (chunk bits 4-5
+// XOR address bits 7-8), and it makes both the per-row writes and the
+// row-group reads of a warp free of bank conflicts.
+__device__ __forceinline__ uint32_t stage_off(int r, int c) {
+  return static_cast<uint32_t>(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+}
+
+// One epilogue warp drains its 32 TMEM lanes (rows q*32 .. q*32+31 of the
+// slab, q = warp % 4 as tcgen05.ld requires) over its half of the BN columns,
+// 32 columns at a time: TMEM -> registers -> scale and cast -> swizzled
+// staging tile in shared memory -> one bulk tensor store (or, for a slab cut
+// by an expert boundary, coalesced row-masked stores).
+template <int BN>
+__device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams& p, const CUtensorMap* tmY,
+                                              uint32_t tmem_acc, int warp, int lane, uint8_t* stage) {
+  static_assert(BN % 64 == 0, "each epilogue warp takes BN/2 columns in chunks of 32");
+  const int q = warp & 3;
+  const int h = (warp - kEpiWarp0) >> 2;
+  const int r = t.row0 + q * 32 + lane;
+  const float sx = r < t.row_end ? __ldg(p.s_x + r) : 0.0f;
+  const uint32_t sbase = smem_u32(stage);
+  const uint32_t taddr0 = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * (BN / 2));
+#pragma unroll 1
+  for (int j = 0; j < BN / 64; ++j) {
+    const int cl = h * (BN / 2) + j * 32;   // first column of the chunk within the tile
+    const int colw = t.n0 + cl + lane;
+    const float sw_lane = colw < p.N ? __ldg(p.s_w + t.sw0 + cl + lane) : 0.0f;
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(taddr0 + static_cast<uint32_t>(j * 32), v);
+    tmem_ld_wait();
+    uint32_t packed[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float w0 = __shfl_sync(0xffffffffu, sw_lane, 2 * i);
+      const float w1 = __shfl_sync(0xffffffffu, sw_lane, 2 * i + 1);
+      const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * i]), sx), w0);
+      const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * i + 1]), sx), w1);
+      const __half2 hv = __floats2half2_rn(y0, y1);
+      packed[i] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    // The previous bulk store of this warp must have finished reading the tile.
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      st_shared_v4(sbase + stage_off(lane, c), packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+    if (t.tma) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmY, stage, t.n0 + cl, t.row0 + q * 32);
+        bulk_commit_group();
+      }
+    } else {
+      __syncwarp();
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int rr = it * 8 + (lane >> 2);
+        const int c = lane & 3;
+        const uint4 val = ld_shared_v4(sbase + stage_off(rr, c));
+        const int grow = t.row0 + q * 32 + rr;
+        const int gcol = t.n0 + cl + c * 8;
+        if (grow < t.row_end && gcol < p.N)
+          *reinterpret_cast<uint4*>(p.Y + static_cast<int64_t>(grow) * p.N + gcol) = val;
+      }
+      __syncwarp();
+    }
+  }
+}
+
+}  // namespace fp8q

@@ -1,5 +1,7 @@
 // FP8 (E4M3 x E4M3) GEMM with FP32 accumulation in tensor memory and a fused
-// per-token x per-channel dequantization + FP16 cast epilogue, for sm_100a.
+// per-token x per-channel dequantization + FP16 cast epilogue, for sm_100a:
+// the single-CTA kernel (128-row tiles), used for the MoE grouped linear and
+// for dense problems of at most 128 rows.
 //
 // Method: "Quantized Inference for OneRec-V2" (关键证据 steps 3-4: FP8 tensor
 // cores, FP32 accumulation, FP16 output) and
@@ -7,19 +9,16 @@
 // Quantize + GEMM + Dequantize; FP8 multiply + FP32 accumulate + FP16 out)
 // and §3.2 (MoE expert GEMMs, pipelined across experts).
 //
-// One persistent kernel serves both the dense linear and the MoE grouped
-// linear.  Each CTA (one per SM) walks output tiles of 128 x BN:
+// Each CTA (one per SM, persistent) walks output tiles of 128 x BN:
 //   warp 0      TMA producer: 128-byte-swizzled 2-D tile loads of A (token
 //               rows, K-major) and B (weight rows, K-major) into a STAGES-deep
 //               shared-memory ring, completion tracked by mbarriers;
 //   warp 1      MMA issuer: one thread issues tcgen05.mma kind::f8f6f4
 //               (M=128, N=BN, K=32 per instruction) into one of two TMEM
-//               accumulators, and tcgen05.commit frees smem stages / hands a
+//               accumulators; tcgen05.commit frees smem stages and hands a
 //               finished accumulator to the epilogue;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
-//               output row per thread), y = fp16((acc * s_x[row]) * s_w[col]),
-//               stores masked by the row limit of the tile (the end of the
-//               expert group for MoE) and by N.
+//   warps 2..9  epilogue (gemm_common.cuh): TMEM -> scale -> fp16 -> bulk
+//               tensor stores, masked at expert-group boundaries.
 // Two TMEM accumulators let the epilogue of tile i overlap the MMAs of tile
 // i+1.  The MoE tile schedule is built on the device from the expert offsets
 // (no host synchronization): tiles are ordered (expert, n-block, m-block), so
@@ -27,28 +26,9 @@
 // it from L2.  No TMA multicast is used anywhere.
 #pragma once
 
-#include <cuda.h>
-
-#include "ptx.cuh"
+#include "gemm_common.cuh"
 
 namespace fp8q {
-
-constexpr int kBM = 128;        // rows of an output tile (TMEM lanes)
-constexpr int kBK = 128;        // K bytes per pipeline stage (one 128-B swizzle row)
-constexpr int kUmmaK = 32;      // K per tcgen05.mma for 8-bit operands
-constexpr int kGemmThreads = 192;
-constexpr int kMaxExperts = 4096;
-
-struct GemmParams {
-  const float* s_x;         // [rows]
-  const float* s_w;         // [E*N]
-  __half* Y;                // [rows, N]
-  const int32_t* offsets;   // [E+1] device, grouped only
-  int rows;                 // M (dense) or total grouped rows
-  int N;
-  int K;
-  int E;                    // 1 for dense
-};
 
 template <int BN, int STAGES>
 struct GemmLayout {
@@ -57,7 +37,7 @@ struct GemmLayout {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kNumBars = 2 * STAGES + 5;   // full, empty, tfull[2], tempty[2], drain
   static constexpr int kTmemCols = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
-  static constexpr int kFixedBytes = STAGES * kStageBytes + kNumBars * 8 + 32;
+  static constexpr int kFixedBytes = STAGES * kStageBytes + kEpiSmemBytes + kNumBars * 8 + 32;
   static size_t smem_bytes(int E) { return 1024 + kFixedBytes + 2 * static_cast<size_t>(E + 1) * 4 + 16; }
 };
 
@@ -74,8 +54,14 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p, int
                                                  const int* tile_prefix, const int* offs) {
   TileCoord c;
   if (!kGrouped) {
-    const int m_blk = t % num_m;
-    const int n_blk = t / num_m;
+    int m_blk, n_blk;
+    if (p.n_fastest) {
+      n_blk = t % num_n;
+      m_blk = t / num_n;
+    } else {
+      m_blk = t % num_m;
+      n_blk = t / num_m;
+    }
     c.a_row0 = m_blk * kBM;
     c.row_end = p.rows;
     c.n0 = n_blk * BN;
@@ -106,9 +92,9 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p, int
 template <int BN, int STAGES, bool kGrouped>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
   using L = GemmLayout<BN, STAGES>;
-  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   constexpr uint32_t kIdesc = idesc_e4m3_f32(kBM, BN);
 
   extern __shared__ uint8_t smem_raw[];
@@ -116,7 +102,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * L::kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * L::kBBytes);
+  uint8_t* sEpi = sB + STAGES * L::kBBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + kEpiSmemBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -141,7 +128,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4 * 32);
+      mbar_init(&tempty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -150,11 +137,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
+  // Inputs (and the expert offsets) may come from the kernel launched just
+  // before this one (programmatic dependent launch): wait for it here, after
+  // the set-up above has overlapped its tail.
+  pdl_wait_prior_grid();
   if (kGrouped) {
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) offs[i] = __ldg(p.offsets + i);
     __syncthreads();
@@ -268,7 +260,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int wq = warp & 3;   // TMEM lane quadrant accessible to this warp
+    uint8_t* stage = sEpi + (warp - kEpiWarp0) * kStageTileBytes;
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -279,43 +271,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int r = c.a_row0 + wq * 32 + lane;
-      const bool valid = r < c.row_end;
-      const float sx = valid ? __ldg(p.s_x + r) : 0.0f;
-      __half* yrow = p.Y + static_cast<int64_t>(valid ? r : 0) * p.N;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(acc * BN);
-#pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(cc * 32), v);
-        tmem_ld_wait();
-        const int col0 = c.n0 + cc * 32;
-        if (valid) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = col0 + q * 8;
-            if (col < p.N) {
-              const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.s_w + c.sw0 + cc * 32 + q * 8));
-              const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.s_w + c.sw0 + cc * 32 + q * 8 + 4));
-              const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-              uint32_t packed[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(v[q * 8 + 2 * i]), sx), w[2 * i]);
-                const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(v[q * 8 + 2 * i + 1]), sx), w[2 * i + 1]);
-                const __half2 h = __floats2half2_rn(y0, y1);
-                packed[i] = *reinterpret_cast<const uint32_t*>(&h);
-              }
-              *reinterpret_cast<uint4*>(yrow + col) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            }
-          }
-        }
-      }
+      EpiTile et;
+      et.row0 = c.a_row0;
+      et.row_end = c.row_end;
+      et.n0 = c.n0;
+      et.sw0 = c.sw0;
+      // A bulk store clips only at the tensor edge, so it is used unless the
+      // slab crosses into the next expert's rows.
+      et.tma = !kGrouped || c.a_row0 + kBM <= c.row_end;
+      epilogue_slab<BN>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage);
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_ph ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   __syncthreads();

@@ -1,0 +1,232 @@
+// FP8 GEMM on CTA pairs (tcgen05 cta_group::2) for the dense linear.
+//
+// Same arithmetic as the single-CTA kernel in gemm_fp8.cuh (E4M3 x E4M3
+// products, FP32 accumulation in TMEM, fused y = fp16((acc * s_x) * s_w);
+// "Quantized Inference for OneRec-V2" 关键证据 steps 3-4;
+// "FP8量化在生成式推荐系统OneRec-V2中的优化实践" §2.3), with the output tile
+// of a cluster of two CTAs = 256 rows x BN columns:
+//   * each CTA stages its own 128 rows of A and BN/2 rows of B per k-block
+//     (32 KB for BN = 256 instead of 48 KB for a 128 x 256 single-CTA tile),
+//     so the same shared memory holds a deeper pipeline and every SM pulls
+//     a third less operand traffic out of L2;
+//   * both CTAs' TMA loads count their bytes on the leader CTA's "full"
+//     mbarrier; the leader's single MMA thread issues the M=256 pair MMA,
+//     whose commits arrive (multicast) on the same barrier in both CTAs;
+//   * each CTA's eight epilogue warps drain their own 128 TMEM lanes
+//     (gemm_common.cuh: bulk tensor stores through a swizzled staging tile)
+//     and arrive on the leader's "accumulator empty" barrier.
+// No TMA multicast: every CTA loads only the tiles it stores.
+#pragma once
+
+#include "gemm_fp8.cuh"
+
+namespace fp8q {
+
+template <int BN, int STAGES>
+struct PairLayout {
+  static constexpr int kABytes = kBM * kBK;            // own 128 rows of A
+  static constexpr int kBRows = BN / 2;                // own half of the B rows
+  static constexpr int kBBytes = kBRows * kBK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kNumBars = 2 * STAGES + 5;      // full, empty, tfull[2], tempty[2], drain
+  static constexpr int kTmemCols = 512;
+  static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes + kEpiSmemBytes + kNumBars * 8 + 32;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+  using L = PairLayout<BN, STAGES>;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256 && (BN / 2) % 8 == 0, "BN");
+  static_assert(2 * BN <= L::kTmemCols, "two accumulators must fit in TMEM");
+  constexpr uint32_t kIdesc = idesc_e4m3_f32(2 * kBM, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * L::kABytes;
+  uint8_t* sEpi = sB + STAGES * L::kBBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + kEpiSmemBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+  const int num_m = (p.rows + 2 * kBM - 1) / (2 * kBM);
+  const int num_n = (p.N + BN - 1) / BN;
+  const int num_kb = (p.K + kBK - 1) / kBK;
+  const int total = num_m * num_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2 * kEpiWarps);   // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, L::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // Both CTAs' barriers are initialized before any cross-CTA arrival or copy.
+  cluster_arrive();
+  cluster_wait();
+  const uint32_t tmem_base = *tmem_slot;
+  // Inputs may come from the kernel launched just before this one.
+  pdl_wait_prior_grid();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const int m_blk = p.n_fastest ? t / num_n : t % num_m;
+        const int n_blk = p.n_fastest ? t % num_n : t / num_m;
+        const int a_row = m_blk * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int b_row = n_blk * BN + static_cast<int>(rank) * L::kBRows;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_leader = mapa_shared(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * L::kStageBytes);
+          tma_load_2d_pair(sA + s * L::kABytes, &tmA, full_leader, kb * kBK, a_row);
+          tma_load_2d_pair(sB + s * L::kBBytes, &tmB, full_leader, kb * kBK, b_row);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        raise_error(0x1u);
+        *abort_flag = 1;
+        // Copies already issued complete within microseconds; let them land
+        // before this CTA's shared memory can be released.
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 50000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader CTA)
+    if (lane == 0 && leader) {
+      int s = 0, acc = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      bool issued = false, ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        if (!mbar_wait(&tempty[acc], acc_ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = sw128_kmajor_desc(smem_u32(sA + s * L::kABytes));
+          const uint64_t b0 = sw128_kmajor_desc(smem_u32(sB + s * L::kBBytes));
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k)
+            mma_f8f6f4_pair(d, a0 + static_cast<uint64_t>(k * kUmmaK / 16),
+                            b0 + static_cast<uint64_t>(k * kUmmaK / 16), kIdesc, (kb | k) != 0 ? 1u : 0u);
+          issued = true;
+          mma_commit_pair_mc(&empty[s], 0x3);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_ph ^= 1u;
+      }
+      if (!ok) {
+        raise_error(0x2u);
+        *abort_flag = 1;
+      }
+      if (issued) {
+        mma_commit_pair_mc(drain, 0x1);
+        mbar_wait(drain, 0, nullptr);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    uint8_t* stage = sEpi + (warp - kEpiWarp0) * kStageTileBytes;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int t = pair; t < total; t += npairs) {
+      const int m_blk = p.n_fastest ? t / num_n : t % num_m;
+      const int n_blk = p.n_fastest ? t % num_n : t / num_m;
+      if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
+        raise_error(0x4u);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      EpiTile et;
+      et.row0 = m_blk * 2 * kBM + static_cast<int>(rank) * kBM;
+      et.row_end = p.rows;
+      et.n0 = n_blk * BN;
+      et.sw0 = et.n0;
+      et.tma = true;   // dense: the bulk store clips at the tensor edge
+      epilogue_slab<BN>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+      acc ^= 1;
+      if (acc == 0) acc_ph ^= 1u;
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+
+  __syncthreads();
+  // The leader has drained its MMAs (which read both CTAs' shared memory) and
+  // all cross-CTA arrivals were issued before this point.
+  tc_fence_before();
+  cluster_arrive();
+  cluster_wait();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace fp8q

@@ -61,6 +61,9 @@ template <int TPR, int VPT>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const __half* __restrict__ X, int M, int K,
                                                         uint8_t* __restrict__ Q, float* __restrict__ S) {
   static_assert(TPR >= 32 && TPR <= 256 && (TPR & (TPR - 1)) == 0, "TPR");
+  // Let a dependent GEMM launched with programmatic serialization start its
+  // set-up now; it waits for this grid's results before reading them.
+  pdl_launch_dependents();
   constexpr int kRowsPerCta = 256 / TPR;
   constexpr int kWarpsPerRow = TPR / 32;
   __shared__ float red[8];
@@ -110,6 +113,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __half* __restric
 __global__ void __launch_bounds__(256) quant_rows_long_kernel(const __half* __restrict__ X, int M, int K,
                                                              uint8_t* __restrict__ Q, float* __restrict__ S) {
   __shared__ float red[8];
+  pdl_launch_dependents();
   const int row = blockIdx.x;
   const int nvec = K >> 3;
   const uint4* src = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(row) * K);

@@ -122,7 +122,7 @@ fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x,
  *   Y_f16 [rows,N] fp16 out: row i of group e = linear of that row with W_e.
  * Empty groups are legal.  Offsets that break the rules are detected on the
  * device: nothing is written and fp8q_device_error() reports
- * FP8Q_DEVERR_BAD_OFFSETS.  E >= 1 and E <= 4096.
+ * FP8Q_DEVERR_BAD_OFFSETS.  E >= 1 and E <= 1024.
  */
 fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x,
                                     const int32_t* offsets, int32_t E, int64_t rows,
@@ -137,6 +137,17 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x,
  * checked against an independent encoder over arbitrary fp32 bit patterns.
  */
 fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* stream);
+
+/*
+ * Tuning override for the dense linear (for measurement and tests; the
+ * defaults are chosen per shape).  kernel_family: 0 = automatic, 1 = the
+ * single-CTA kernel (128-row tiles), 2 = the CTA-pair kernel (256-row tiles,
+ * tcgen05 cta_group::2).  tile_n: 0 = automatic, else 128, 192 or 256 (pair
+ * kernel only).  Process-wide; not thread-safe against concurrent launches.
+ * Environment variables FP8Q_FORCE_KERNEL (auto|single|pair) and FP8Q_BN set
+ * the initial values.
+ */
+fp8q_status fp8q_set_gemm_tuning(int kernel_family, int tile_n);
 
 /*
  * Synchronizes `stream`, then reads and clears the device error word of the

@@ -81,7 +81,7 @@ def test_linear_zero_rows_is_noop(L):
 
 
 @pytest.mark.parametrize("E,rows,N,K,off", [
-    (0, 8, 16, 32, 0x1000), (4097, 8, 16, 32, 0x1000), (4, 8, 12, 32, 0x1000),
+    (0, 8, 16, 32, 0x1000), (1025, 8, 16, 32, 0x1000), (4, 8, 12, 32, 0x1000),
     (4, 8, 16, 20, 0x1000), (4, 8, 16, 32, 0), (4, 8, 16, 32, 0x1002), (4, -1, 16, 32, 0x1000),
 ])
 def test_moe_rejects(L, E, rows, N, K, off):

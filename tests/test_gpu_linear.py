@@ -107,3 +107,18 @@ def test_zero_rows_noop(fq):
     sw = torch.ones((64,), dtype=torch.float32, device="cuda")
     Y = fq.linear(Xq, s, Wq, sw)
     assert Y.shape == (0, 64)
+
+
+VARIANTS = [(1, 0), (2, 128), (2, 192), (2, 256)]
+
+
+@pytest.mark.parametrize("family,bn", VARIANTS)
+@pytest.mark.parametrize("M,N,K", [(300, 520, 272), (257, 1000, 1040), (1024, 6144, 2048), (512, 768, 128)])
+def test_kernel_variants(fq, family, bn, M, N, K):
+    X = wl.random_f16((M, K), seed=M + 3 * N + K)
+    W = wl.random_f16((N, K), seed=N + K, std=0.02)
+    fq.set_gemm_tuning(family, bn)
+    try:
+        check(fq, X, W, what=f"family={family} bn={bn} {M}x{N}x{K}")
+    finally:
+        fq.set_gemm_tuning(0, 0)

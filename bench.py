@@ -145,7 +145,6 @@ class Plan:
         self.fq, self.L = fq, _lib
         self.kind = kind
         self.device = device
-        self.stream = torch.cuda.current_stream(device).cuda_stream
         if kind == "dense":
             X, W = tensors
             self.M, self.K = X.shape
@@ -207,7 +206,8 @@ class Plan:
 
     def launch(self, i, k):
         """Launch kernel k of step i (raw C ABI, integer pointers)."""
-        L, p, st = self.L, self.bufs[i % self.sets]["p"], self.stream
+        L, p = self.L, self.bufs[i % self.sets]["p"]
+        st = torch.cuda.current_stream(self.device).cuda_stream   # the capture stream inside a graph
         if self.kind == "dense":
             if k == 0:
                 s = L.fp8q_quantize_rows_dynamic(p["X"], self.M, self.K, p["Xq"], p["sx"], st)
@@ -232,29 +232,72 @@ class Plan:
             self.launch(i, k)
 
 
-def timed_gpu(plan, steps, warmup, barrier):
+def _graph_of(plan, launches):
+    """Capture the (step, kernel) launches into a CUDA graph and upload it."""
     dev = plan.device
-    for i in range(warmup):
-        plan.step(i)
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(device=dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.graph(g, stream=cap):
+        for i, k in launches:
+            plan.launch(i, k)
     torch.cuda.synchronize(dev)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    return g
+
+
+def timed_gpu(plan, steps, barrier, use_graph=True):
+    """Time exactly `steps` steps of the path.
+
+    With use_graph the steps are captured once into a CUDA graph (launch
+    overhead removed, as a serving loop would run them); the graph is
+    replayed once untimed to upload it, then the timed replay is bracketed by
+    CUDA events on the replay stream.  Each kernel's own duration is timed the
+    same way from a graph holding only that kernel's launches of the same
+    steps (events recorded inside a graph cannot be timed).
+    """
+    dev = plan.device
     nk = plan.launches_per_step
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
-          for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if not use_graph:
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+              for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        t0.record()
+        for i in range(steps):
+            for k in range(nk):
+                ev[i][k][0].record()
+                plan.launch(i, k)
+                ev[i][k][1].record()
+        t1.record()
+        torch.cuda.synchronize(dev)
+        barrier()
+        per_kernel_ms = [statistics.fmean(ev[i][k][0].elapsed_time(ev[i][k][1]) for i in range(steps))
+                         for k in range(nk)]
+        return t0.elapsed_time(t1), per_kernel_ms
+
+    g = _graph_of(plan, [(i, k) for i in range(steps) for k in range(nk)])
     barrier()
     torch.cuda.synchronize(dev)
     t0.record()
-    for i in range(steps):
-        for k in range(nk):
-            ev[i][k][0].record()
-            plan.launch(warmup + i, k)
-            ev[i][k][1].record()
+    g.replay()
     t1.record()
     torch.cuda.synchronize(dev)
     barrier()
     total_ms = t0.elapsed_time(t1)
-    per_kernel_ms = [statistics.fmean(ev[i][k][0].elapsed_time(ev[i][k][1]) for i in range(steps))
-                     for k in range(nk)]
+    del g
+    per_kernel_ms = []
+    for k in range(nk):
+        gk = _graph_of(plan, [(i, k) for i in range(steps)])
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        gk.replay()
+        b.record()
+        torch.cuda.synchronize(dev)
+        per_kernel_ms.append(a.elapsed_time(b) / steps)
+        del gk
     return total_ms, per_kernel_ms
 
 
@@ -415,7 +458,7 @@ def run_ours(args, world, rank, local):
     barrier = make_barrier(world, device)
     desc, kind, tensors = workload_spec(args.workload)
     import fp8_quantized_generative_b200 as fq
-    fq.set_gemm_tuning({"auto": 0, "single": 1, "pair": 2}[args.gemm], args.bn)
+    fq.set_gemm_tuning({"auto": 0, "single": 1, "pair": 2, "splitk": 3}[args.gemm], args.bn, args.ksplit)
     plan = Plan(kind, tensors, device, min_rotation_bytes=3 * L2_BYTES)
     peaks, peak_src = load_peaks()
 
@@ -425,7 +468,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(device)
     sampler.start()
     time.sleep(0.2)
-    total_ms, per_kernel_ms = timed_gpu(plan, args.steps, 0, barrier)
+    total_ms, per_kernel_ms = timed_gpu(plan, args.steps, barrier, use_graph=not args.no_graph)
     clocks = sampler.stop()
     flag = plan.fq.device_error()
     if flag:
@@ -471,10 +514,14 @@ def run_ours(args, world, rank, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3 (fp32 accumulate, fp16 out)",
             "data": "synthetic",
             "config": {"workload": desc, "parallelism": f"replicas x{world} (no collective)",
-                       "gemm": args.gemm, "bn": args.bn,
+                       "gemm": args.gemm, "bn": args.bn, "ksplit": args.ksplit,
                        "l2": f"rotating {plan.sets} buffer sets of {plan.bytes_per_set / 1e6:.0f} MB "
                              f"(> 3x 126 MB L2), no flush",
-                       "step": " -> ".join(plan.kernels)},
+                       "step": " -> ".join(plan.kernels),
+                       "launch": "per-call from the host" if args.no_graph else
+                                 "CUDA graph of the K timed steps (replayed once untimed to upload)",
+                       "kernel_timing": "per-kernel: CUDA events around a graph of that kernel's K launches"
+                                        if not args.no_graph else "per-kernel: CUDA events around each launch"},
             "roofline": roofline, "kernels": kern,
             "step_gb_s": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
             "pct_fp8_peak_step": round(100 * step_flops / (ms_step * 1e-3) / 1e12 / fp8_peak, 2),
@@ -505,9 +552,11 @@ def main(argv=None):
     ap.add_argument("--workload", default="qkv")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--gemm", default="auto", choices=["auto", "single", "pair"],
+    ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of a CUDA graph")
+    ap.add_argument("--gemm", default="auto", choices=["auto", "single", "pair", "splitk"],
                     help="dense GEMM kernel family (tuning sweeps; default: chosen per shape)")
     ap.add_argument("--bn", type=int, default=0, help="pair-kernel tile width (0 = automatic)")
+    ap.add_argument("--ksplit", type=int, default=0, help="split-K cluster size for M <= 128 (0 = automatic)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

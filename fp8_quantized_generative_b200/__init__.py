@@ -118,9 +118,9 @@ def e4m3_encode_f32(x: torch.Tensor) -> torch.Tensor:
     return out
 
 
-def set_gemm_tuning(kernel_family: int = 0, tile_n: int = 0) -> None:
+def set_gemm_tuning(kernel_family: int = 0, tile_n: int = 0, ksplit: int = 0) -> None:
     """Override the dense-linear kernel choice (0 = automatic; see include/fp8q.h)."""
-    check(_lib.fp8q_set_gemm_tuning(kernel_family, tile_n), "fp8q_set_gemm_tuning")
+    check(_lib.fp8q_set_gemm_tuning(kernel_family, tile_n, ksplit), "fp8q_set_gemm_tuning")
 
 
 def device_error(device=None) -> int:

@@ -47,7 +47,7 @@ SIGNATURES = {
     "fp8q_linear": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "fp8q_moe_grouped_linear": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_e4m3_encode_f32": (_INT, [_P, _I64, _P, _P]),
-    "fp8q_set_gemm_tuning": (_INT, [_INT, _INT]),
+    "fp8q_set_gemm_tuning": (_INT, [_INT, _INT, _INT]),
     "fp8q_device_error": (_INT, [_P, ctypes.POINTER(ctypes.c_uint32)]),
 }
 
@@ -108,8 +108,8 @@ def fp8q_e4m3_encode_f32(x, n, out, stream):
     return lib().fp8q_e4m3_encode_f32(x, n, out, stream)
 
 
-def fp8q_set_gemm_tuning(kernel_family, tile_n):
-    return lib().fp8q_set_gemm_tuning(kernel_family, tile_n)
+def fp8q_set_gemm_tuning(kernel_family, tile_n, ksplit=0):
+    return lib().fp8q_set_gemm_tuning(kernel_family, tile_n, ksplit)
 
 
 def fp8q_device_error(stream):

@@ -15,6 +15,7 @@
 #include "fp8q.h"
 #include "gemm_fp8.cuh"
 #include "gemm_fp8_pair.cuh"
+#include "gemm_fp8_splitk.cuh"
 #include "quant_rows.cuh"
 
 namespace fp8q {
@@ -134,8 +135,9 @@ constexpr int kStages = 4;
 //   FP8Q_BN           = 0 (auto) | 128 | 192 | 256   (pair-kernel tile width)
 // fp8q_set_gemm_tuning() overrides both at run time.
 struct Knobs {
-  int force = 0;  // 0 auto, 1 single, 2 pair
+  int force = 0;  // 0 auto, 1 single, 2 pair, 3 split-K (M <= 128)
   int bn = 0;
+  int ksplit = 0; // split-K cluster size, 0 = automatic
 };
 Knobs& knobs() {
   static Knobs k = []() {
@@ -143,11 +145,26 @@ Knobs& knobs() {
     if (const char* f = std::getenv("FP8Q_FORCE_KERNEL")) {
       if (!std::strcmp(f, "single")) r.force = 1;
       if (!std::strcmp(f, "pair")) r.force = 2;
+      if (!std::strcmp(f, "splitk")) r.force = 3;
     }
+    if (const char* k = std::getenv("FP8Q_KSPLIT")) r.ksplit = std::atoi(k);
     if (const char* b = std::getenv("FP8Q_BN")) r.bn = std::atoi(b);
     return r;
   }();
   return k;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute
+// persists; setting it on every call would cost a driver round trip).
+template <auto Kernel>
+cudaError_t ensure_smem(size_t bytes, int dev) {
+  static bool done[kMaxDevices] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  if (done[dev]) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
 }
 
 template <typename... Args>
@@ -194,7 +211,7 @@ fp8q_status launch_gemm(const uint8_t* A, int64_t a_rows, const uint8_t* B, int6
   if (s != FP8Q_OK) return s;
   auto kernel = fp8_gemm_kernel<kBN, kStages, kGrouped>;
   const size_t smem = L::smem_bytes(kGrouped ? p.E : 0);
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  e = ensure_smem<fp8_gemm_kernel<kBN, kStages, kGrouped>>(L::smem_bytes(kGrouped ? kMaxExperts : 0), dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   const int grid = static_cast<int>(tiles_upper_bound < sms ? (tiles_upper_bound < 1 ? 1 : tiles_upper_bound) : sms);
   e = launch_ex(kernel, dim3(grid), dim3(kGemmThreads), smem, st, 1, true, ta, tb, ty, p);
@@ -211,7 +228,10 @@ int max_pair_clusters(int dev) {
   if (cache[dev] > 0) return cache[dev];
   using L = PairLayout<BN, STAGES>;
   auto kernel = fp8_gemm_pair_kernel<BN, STAGES>;
-  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L::kSmemBytes));
+  if (ensure_smem<fp8_gemm_pair_kernel<BN, STAGES>>(L::kSmemBytes, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2);
   cfg.blockDim = dim3(kGemmThreads);
@@ -244,8 +264,7 @@ fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, const GemmParams& p,
   s = make_output_map(&ty, p.Y, p.rows, p.N);
   if (s != FP8Q_OK) return s;
   auto kernel = fp8_gemm_pair_kernel<BN, STAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(L::kSmemBytes));
+  cudaError_t e = ensure_smem<fp8_gemm_pair_kernel<BN, STAGES>>(L::kSmemBytes, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair)");
   const int clusters = max_pair_clusters<BN, STAGES>(dev);
   if (clusters < 1) {
@@ -284,11 +303,87 @@ int choose_pair_bn(int64_t M, int64_t N, int clusters) {
   return best;
 }
 
+// How many clusters of S CTAs of a split-K kernel fit on the device at once.
+template <int MPAD, int STAGES>
+int max_splitk_clusters(int dev, int S) {
+  static int cache[kMaxDevices][9] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  if (cache[dev][S] != 0) return cache[dev][S];
+  using L = SplitKLayout<MPAD, STAGES>;
+  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES>;
+  if (ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES>>(L::kSmemBytes, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S);
+  cfg.blockDim = dim3(kSkThreads);
+  cfg.dynamicSmemBytes = L::kSmemBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = S;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    n = -1;
+  }
+  cache[dev][S] = n;
+  return n;
+}
+
+// Split factor: as many CTAs per 128-channel weight tile as keeps every
+// cluster of the grid resident at once (one wave), at most 8 and at most the
+// number of K blocks.
+template <int MPAD, int STAGES>
+int choose_ksplit(int dev, int sms, int n_tiles, int num_kb) {
+  int S = n_tiles > 0 ? sms / n_tiles : 1;
+  if (S > 8) S = 8;
+  if (S > num_kb) S = num_kb;
+  if (S < 1) S = 1;
+  while (S > 1) {
+    const int fit = max_splitk_clusters<MPAD, STAGES>(dev, S);
+    if (fit >= n_tiles) break;
+    --S;
+  }
+  return S;
+}
+
+template <int MPAD, int STAGES>
+fp8q_status launch_splitk(const uint8_t* Xq, const uint8_t* Wq, const GemmParams& p, int dev, int sms,
+                          cudaStream_t st) {
+  using L = SplitKLayout<MPAD, STAGES>;
+  CUtensorMap tw, tx;
+  fp8q_status s = make_operand_map(&tw, Wq, p.N, p.K, kBM);
+  if (s != FP8Q_OK) return s;
+  s = make_operand_map(&tx, Xq, p.rows, p.K, MPAD);
+  if (s != FP8Q_OK) return s;
+  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES>;
+  cudaError_t e = ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES>>(L::kSmemBytes, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(splitk)");
+  const int n_tiles = (p.N + kBM - 1) / kBM;
+  const int num_kb = (p.K + kBK - 1) / kBK;
+  const int S = knobs().ksplit ? knobs().ksplit : choose_ksplit<MPAD, STAGES>(dev, sms, n_tiles, num_kb);
+  e = launch_ex(kernel, dim3(n_tiles * S), dim3(kSkThreads), L::kSmemBytes, st, S, true, tw, tx, p);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_splitk_kernel launch");
+  return FP8Q_OK;
+}
+
 fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams& p, cudaStream_t st) {
   int dev = 0, sms = 0;
   cudaError_t e = current_device_info(&dev, &sms);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
   const Knobs kn = knobs();
+  if ((kn.force == 0 && p.rows <= kBM) || kn.force == 3) {
+    if (p.rows <= 16) return launch_splitk<16, 10>(Xq, Wq, p, dev, sms, st);
+    if (p.rows <= 32) return launch_splitk<32, 9>(Xq, Wq, p, dev, sms, st);
+    if (p.rows <= 64) return launch_splitk<64, 8>(Xq, Wq, p, dev, sms, st);
+    if (p.rows <= 128) return launch_splitk<128, 6>(Xq, Wq, p, dev, sms, st);
+  }
   bool pair = p.rows > kBM;
   // Walk n-blocks first when A is the larger operand: each A block is then
   // reused by every n-block while it is in L2, and the smaller B stays there.
@@ -424,11 +519,13 @@ fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* 
   return FP8Q_OK;
 }
 
-fp8q_status fp8q_set_gemm_tuning(int kernel_family, int tile_n) {
-  if (kernel_family < 0 || kernel_family > 2) return invalid("kernel_family must be 0, 1 or 2");
+fp8q_status fp8q_set_gemm_tuning(int kernel_family, int tile_n, int ksplit) {
+  if (kernel_family < 0 || kernel_family > 3) return invalid("kernel_family must be 0, 1, 2 or 3");
   if (tile_n != 0 && tile_n != 128 && tile_n != 192 && tile_n != 256) return invalid("tile_n must be 0, 128, 192 or 256");
+  if (ksplit < 0 || ksplit > 8) return invalid("ksplit must be in [0, 8]");
   knobs().force = kernel_family;
   knobs().bn = tile_n;
+  knobs().ksplit = ksplit;
   return FP8Q_OK;
 }
 

@@ -310,3 +310,17 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 }
 
 }  // namespace fp8q
+
+namespace fp8q {
+// 32-bit load from (possibly another CTA's) shared memory, shared::cluster address.
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+}  // namespace fp8q

@@ -121,4 +121,17 @@ def test_kernel_variants(fq, family, bn, M, N, K):
     try:
         check(fq, X, W, what=f"family={family} bn={bn} {M}x{N}x{K}")
     finally:
-        fq.set_gemm_tuning(0, 0)
+        fq.set_gemm_tuning(0, 0, 0)
+
+
+@pytest.mark.parametrize("ksplit", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (5, 264, 272), (16, 1000, 2048), (33, 520, 1040),
+                                   (64, 256, 128), (100, 6144, 2048), (128, 4096, 4096)])
+def test_splitk_variants(fq, ksplit, M, N, K):
+    X = wl.random_f16((M, K), seed=7 * M + N + K)
+    W = wl.random_f16((N, K), seed=N + 2 * K, std=0.02)
+    fq.set_gemm_tuning(3, 0, ksplit)
+    try:
+        check(fq, X, W, what=f"splitk S={ksplit} {M}x{N}x{K}")
+    finally:
+        fq.set_gemm_tuning(0, 0, 0)

@@ -127,8 +127,10 @@ fp8q_status make_output_map(CUtensorMap* m, const void* base, int64_t rows, int6
 }
 
 // ------------------------------------------------------------------ GEMM launch
-constexpr int kBN = 256;
+constexpr int kBN = 256;        // single-CTA dense tiles (128 x 256)
 constexpr int kStages = 4;
+constexpr int kBNGrouped = 256; // MoE tiles (128 x 256); 128-wide tiles measured slower on B200
+constexpr int kStagesGrouped = 4;
 
 // Tuning knobs read once from the environment (for measurement sweeps):
 //   FP8Q_FORCE_KERNEL = auto | single | pair   (dense linear kernel family)
@@ -197,21 +199,23 @@ cudaError_t launch_ex(void (*kernel)(Args...), dim3 grid, dim3 block, size_t sme
 template <bool kGrouped>
 fp8q_status launch_gemm(const uint8_t* A, int64_t a_rows, const uint8_t* B, int64_t b_rows, const GemmParams& p,
                         int64_t tiles_upper_bound, cudaStream_t st) {
-  using L = GemmLayout<kBN, kStages>;
+  constexpr int BN = kGrouped ? kBNGrouped : kBN;
+  constexpr int STAGES = kGrouped ? kStagesGrouped : kStages;
+  using L = GemmLayout<BN, STAGES>;
   int dev = 0, sms = 0;
   cudaError_t e = current_device_info(&dev, &sms);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
   CUtensorMap ta, tb;
   fp8q_status s = make_operand_map(&ta, A, a_rows, p.K, kBM);
   if (s != FP8Q_OK) return s;
-  s = make_operand_map(&tb, B, b_rows, p.K, kBN);
+  s = make_operand_map(&tb, B, b_rows, p.K, BN);
   if (s != FP8Q_OK) return s;
   CUtensorMap ty;
   s = make_output_map(&ty, p.Y, p.rows, p.N);
   if (s != FP8Q_OK) return s;
-  auto kernel = fp8_gemm_kernel<kBN, kStages, kGrouped>;
+  auto kernel = fp8_gemm_kernel<BN, STAGES, kGrouped>;
   const size_t smem = L::smem_bytes(kGrouped ? p.E : 0);
-  e = ensure_smem<fp8_gemm_kernel<kBN, kStages, kGrouped>>(L::smem_bytes(kGrouped ? kMaxExperts : 0), dev);
+  e = ensure_smem<fp8_gemm_kernel<BN, STAGES, kGrouped>>(L::smem_bytes(kGrouped ? kMaxExperts : 0), dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   const int grid = static_cast<int>(tiles_upper_bound < sms ? (tiles_upper_bound < 1 ? 1 : tiles_upper_bound) : sms);
   e = launch_ex(kernel, dim3(grid), dim3(kGemmThreads), smem, st, 1, true, ta, tb, ty, p);
@@ -339,16 +343,18 @@ int max_splitk_clusters(int dev, int S) {
 // Split factor: as many CTAs per 128-channel weight tile as keeps every
 // cluster of the grid resident at once (one wave), at most 8 and at most the
 // number of K blocks.
+// Split factor S in {1, 2, 4, 8} (a divisor of the 128 weight rows of a
+// tile, so each CTA of the cluster owns an equal slice of the reduction):
+// the largest that keeps every cluster of the grid resident at once (one
+// wave) and gives each CTA at least one K block.
 template <int MPAD, int STAGES>
 int choose_ksplit(int dev, int sms, int n_tiles, int num_kb) {
-  int S = n_tiles > 0 ? sms / n_tiles : 1;
-  if (S > 8) S = 8;
-  if (S > num_kb) S = num_kb;
-  if (S < 1) S = 1;
+  int S = 8;
+  while (S > 1 && (n_tiles * S > sms || S > num_kb)) S >>= 1;
   while (S > 1) {
     const int fit = max_splitk_clusters<MPAD, STAGES>(dev, S);
     if (fit >= n_tiles) break;
-    --S;
+    S >>= 1;
   }
   return S;
 }
@@ -379,10 +385,13 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
   if (e != cudaSuccess) return cuda_fail(e, "device query");
   const Knobs kn = knobs();
   if ((kn.force == 0 && p.rows <= kBM) || kn.force == 3) {
-    if (p.rows <= 16) return launch_splitk<16, 10>(Xq, Wq, p, dev, sms, st);
-    if (p.rows <= 32) return launch_splitk<32, 9>(Xq, Wq, p, dev, sms, st);
-    if (p.rows <= 64) return launch_splitk<64, 8>(Xq, Wq, p, dev, sms, st);
-    if (p.rows <= 128) return launch_splitk<128, 6>(Xq, Wq, p, dev, sms, st);
+    // Up to 64 rows the stage count keeps shared memory under half an SM
+    // (two CTAs resident), so the CTAs of the next kernel on the stream can
+    // start and prefetch their weights while this one drains.
+    if (p.rows <= 16) return launch_splitk<16, 5>(Xq, Wq, p, dev, sms, st);
+    if (p.rows <= 32) return launch_splitk<32, 4>(Xq, Wq, p, dev, sms, st);
+    if (p.rows <= 64) return launch_splitk<64, 3>(Xq, Wq, p, dev, sms, st);
+    if (p.rows <= 128) return launch_splitk<128, 4>(Xq, Wq, p, dev, sms, st);
   }
   bool pair = p.rows > kBM;
   // Walk n-blocks first when A is the larger operand: each A block is then
@@ -499,7 +508,7 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const i
   p.K = static_cast<int>(K);
   p.E = E;
   p.n_fastest = 0;
-  const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBN - 1) / kBN);
+  const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBNGrouped - 1) / kBNGrouped);
   return launch_gemm<true>(Xq, rows, Wq, int64_t(E) * N, p, tiles, static_cast<cudaStream_t>(stream));
 }
 
@@ -522,7 +531,8 @@ fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* 
 fp8q_status fp8q_set_gemm_tuning(int kernel_family, int tile_n, int ksplit) {
   if (kernel_family < 0 || kernel_family > 3) return invalid("kernel_family must be 0, 1, 2 or 3");
   if (tile_n != 0 && tile_n != 128 && tile_n != 192 && tile_n != 256) return invalid("tile_n must be 0, 128, 192 or 256");
-  if (ksplit < 0 || ksplit > 8) return invalid("ksplit must be in [0, 8]");
+  if (ksplit != 0 && ksplit != 1 && ksplit != 2 && ksplit != 4 && ksplit != 8)
+    return invalid("ksplit must be 0, 1, 2, 4 or 8");
   knobs().force = kernel_family;
   knobs().bn = tile_n;
   knobs().ksplit = ksplit;

@@ -171,6 +171,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = *total_s;
+  // The next kernel on the stream may begin launching (it waits for this
+  // grid before touching anything this grid reads or writes).
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer

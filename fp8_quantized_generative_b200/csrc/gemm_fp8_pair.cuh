@@ -97,8 +97,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cluster_arrive();
   cluster_wait();
   const uint32_t tmem_base = *tmem_slot;
-  // Inputs may come from the kernel launched just before this one.
-  pdl_wait_prior_grid();
+  // The next kernel on the stream may begin launching (it waits for this
+  // grid before touching anything this grid reads or writes).
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -106,12 +107,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      // The weights do not depend on the kernel launched before this one
+      // (programmatic dependent launch): request the first ring pass of the
+      // first tile's weight tiles before waiting for it; only the activation
+      // tiles wait.
+      int pre = 0;
+      if (pair < total) {
+        const int n_blk = p.n_fastest ? pair % num_n : pair / num_m;
+        const int b_row = n_blk * BN + static_cast<int>(rank) * L::kBRows;
+        pre = num_kb < STAGES ? num_kb : STAGES;
+        for (int i = 0; i < pre; ++i) {
+          const uint32_t full_leader = mapa_shared(smem_u32(&full[i]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[i], 2 * L::kStageBytes);
+          tma_load_2d_pair(sB + i * L::kBBytes, &tmB, full_leader, i * kBK, b_row);
+        }
+      }
+      pdl_wait_prior_grid();
       for (int t = pair; t < total && ok; t += npairs) {
         const int m_blk = p.n_fastest ? t / num_n : t % num_m;
         const int n_blk = p.n_fastest ? t % num_n : t / num_m;
         const int a_row = m_blk * 2 * kBM + static_cast<int>(rank) * kBM;
         const int b_row = n_blk * BN + static_cast<int>(rank) * L::kBRows;
         for (int kb = 0; kb < num_kb; ++kb) {
+          if (pre > 0) {
+            // stage kb of the first pass: weights already requested
+            const uint32_t full_leader = mapa_shared(smem_u32(&full[s]), 0);
+            tma_load_2d_pair(sA + s * L::kABytes, &tmA, full_leader, kb * kBK, a_row);
+            --pre;
+            if (++s == STAGES) {
+              s = 0;
+              ph ^= 1u;
+            }
+            continue;
+          }
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -139,6 +167,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader CTA)
+    pdl_wait_prior_grid();
     if (lane == 0 && leader) {
       int s = 0, acc = 0;
       uint32_t ph = 0, acc_ph = 0;
@@ -186,6 +215,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    pdl_wait_prior_grid();   // s_x comes from, and Y may be read by, the neighbouring kernels
     uint8_t* stage = sEpi + (warp - kEpiWarp0) * kStageTileBytes;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);

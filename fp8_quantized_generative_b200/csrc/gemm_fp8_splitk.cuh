@@ -12,10 +12,14 @@
 //     operand, so a single token still uses a full-height MMA;
 //   * the S CTAs of a cluster (cluster dims (S,1,1)) each take 1/S of the K
 //     blocks and accumulate a 128 x MPAD fp32 partial in TMEM;
-//   * every CTA copies its partial into its own shared memory, the cluster
-//     synchronizes, and CTA r sums lanes [r*128/S, (r+1)*128/S) of all S
-//     partials (ranks in fixed order 0..S-1, so results are reproducible),
-//     applies the scales and writes fp16 -- no global scratch memory.
+//   * S is 1, 2, 4 or 8; every CTA pushes the rows of its partial that CTA
+//     r owns (rows [r*128/S, (r+1)*128/S)) into CTA r's receive buffer with
+//     st.shared::cluster; after one cluster barrier CTA r sums its S slices
+//     locally in fixed rank order 0..S-1 (reproducible), applies the scales
+//     and writes fp16 -- no global scratch memory, no remote loads;
+//   * the weight tiles do not depend on the kernel launched before this one,
+//     so the first STAGES of them are requested before the programmatic-
+//     dependent-launch wait: their DRAM latency overlaps that kernel's tail.
 #pragma once
 
 #include "gemm_common.cuh"
@@ -29,13 +33,15 @@ struct SplitKLayout {
   static constexpr int kWBytes = kBM * kBK;            // 128 weight rows x 128 K bytes
   static constexpr int kXBytes = MPAD * kBK;           // MPAD token rows
   static constexpr int kStageBytes = kWBytes + kXBytes;
-  static constexpr int kPitch = MPAD + 1;              // fp32 words per partial row (odd: no bank conflicts)
-  static constexpr int kPartialBytes = kBM * kPitch * 4;
   static constexpr int kRingBytes = STAGES * kStageBytes;
-  static constexpr int kBodyBytes = kRingBytes > kPartialBytes ? kRingBytes : kPartialBytes;
+  // Receive buffer: [S][128/S rows][MPAD + 4] fp32 = 128 rows of MPAD + 4
+  // words (16-byte aligned rows; the +4 keeps 8 consecutive rows of a
+  // 16-byte access on distinct bank groups).
+  static constexpr int kPitch = MPAD + 4;
+  static constexpr int kRecvBytes = kBM * kPitch * 4;
   static constexpr int kNumBars = 2 * STAGES + 2;      // full, empty, tfull, drain
   static constexpr int kTmemCols = MPAD < 32 ? 32 : MPAD;
-  static constexpr size_t kSmemBytes = 1024 + size_t(kBodyBytes) + kNumBars * 8 + 32;
+  static constexpr size_t kSmemBytes = 1024 + size_t(kRingBytes) + kRecvBytes + kNumBars * 8 + 32;
 };
 
 template <int MPAD, int STAGES>
@@ -51,8 +57,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sW = smem;
   uint8_t* sX = smem + STAGES * L::kWBytes;
-  float* part = reinterpret_cast<float*>(smem);   // reused after the mainloop
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBodyBytes);
+  float* recv = reinterpret_cast<float*>(smem + L::kRingBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kRingBytes + L::kRecvBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -71,6 +77,11 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   const int kb1 = static_cast<int>((int64_t(rank + 1) * num_kb) / S);
   const int nkb = kb1 - kb0;
 
+  // Thread 0 is also the producer: it initializes the barriers and at once
+  // requests the weight tiles of the first ring pass.  The weights do not
+  // depend on the kernel launched before this one (programmatic dependent
+  // launch), so their DRAM latency overlaps that kernel and this set-up.
+  const int pre = nkb < STAGES ? nkb : STAGES;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -80,9 +91,10 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmW);
+    for (int i = 0; i < pre; ++i) {
+      mbar_arrive_expect_tx(&full[i], L::kStageBytes);
+      tma_load_2d(sW + i * L::kWBytes, &tmW, &full[i], (kb0 + i) * kBK, n0);
+    }
     prefetch_tmap(&tmX);
   }
   if (warp == 1) {
@@ -93,13 +105,23 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait_prior_grid();
+  // The next kernel on the stream may begin launching (it waits for this
+  // grid before touching anything this grid reads or writes).
+  pdl_launch_dependents();
+  // Every CTA of the cluster must be running before any pushes into its
+  // shared memory: arrive now, wait just before the first remote access.
+  cluster_arrive_relaxed();
 
   if (warp == 0) {
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0, armed = 0, armed_ph = 0;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      // The first ring pass of weight tiles is already in flight; the token
+      // rows come from the previous kernel.
+      pdl_wait_prior_grid();
+      for (int i = 0; i < pre; ++i) tma_load_2d(sX + i * L::kXBytes, &tmX, &full[i], (kb0 + i) * kBK, 0);
+      int s = pre % STAGES;
+      uint32_t ph = pre == STAGES ? 1u : 0u;
+      uint32_t armed = pre == STAGES ? (1u << STAGES) - 1u : (1u << pre) - 1u, armed_ph = 0;
+      for (int kb = kb0 + pre; kb < kb1; ++kb) {
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
           raise_error(0x1u);
           *abort_flag = 1;
@@ -119,7 +141,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         if (armed & (1u << i)) mbar_wait(&full[i], (armed_ph >> i) & 1u, nullptr);
     }
     __syncwarp();
+    cluster_wait();
   } else if (warp == 1) {
+    pdl_wait_prior_grid();
     if (lane == 0 && nkb > 0) {
       int s = 0;
       uint32_t ph = 0;
@@ -149,11 +173,15 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       mbar_wait(drain, 0, nullptr);
     }
     __syncwarp();
+    cluster_wait();
   } else {
-    // Partial (TMEM lanes = weight rows of the tile, columns = token rows)
-    // -> own shared memory, row pitch MPAD + 1 words.
+    pdl_wait_prior_grid();
+    // Partial: TMEM lane = weight row n of the tile, column = token row m.
+    // Row n belongs to CTA n / SL of the cluster, which receives it at slot
+    // [this rank][n % SL] of its receive buffer.
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int SL = kBM / S;
     bool have = nkb > 0;
     if (have && !mbar_wait(tfull, 0, abort_flag)) {
       raise_error(0x4u);
@@ -161,62 +189,78 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       have = false;
     }
     tc_fence_after();
-    float* prow = part + row * L::kPitch;
-    if (have) {
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      if (MPAD == 16) {
-        uint32_t v[16];
+    cluster_wait();
+    const int owner = row / SL;
+    const uint32_t dst = mapa_shared(smem_u32(recv + (rank * SL + row % SL) * L::kPitch), static_cast<uint32_t>(owner));
+    const int mcols = (p.rows + 3) & ~3;   // token rows actually needed, rounded to 4
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    if (MPAD == 16) {
+      uint32_t v[16];
+      if (have) {
         tmem_ld_32x32b_x16(taddr, v);
         tmem_ld_wait();
+      }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) prow[i] = __uint_as_float(v[i]);
-      } else {
+      for (int i = 0; i < 16; i += 4)
+        if (i < mcols)
+          st_dsmem_v4(dst + i * 4, have ? __uint_as_float(v[i]) : 0.f, have ? __uint_as_float(v[i + 1]) : 0.f,
+                      have ? __uint_as_float(v[i + 2]) : 0.f, have ? __uint_as_float(v[i + 3]) : 0.f);
+    } else {
 #pragma unroll 1
-        for (int c = 0; c < MPAD / 32; ++c) {
-          uint32_t v[32];
+      for (int c = 0; c < MPAD / 32; ++c) {
+        if (c * 32 >= mcols) break;
+        uint32_t v[32];
+        if (have) {
           tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
           tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) prow[c * 32 + i] = __uint_as_float(v[i]);
         }
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          if (c * 32 + i < mcols)
+            st_dsmem_v4(dst + (c * 32 + i) * 4, have ? __uint_as_float(v[i]) : 0.f,
+                        have ? __uint_as_float(v[i + 1]) : 0.f, have ? __uint_as_float(v[i + 2]) : 0.f,
+                        have ? __uint_as_float(v[i + 3]) : 0.f);
       }
-    } else {
-      for (int i = 0; i < MPAD; ++i) prow[i] = 0.0f;
     }
     tc_fence_before();
   }
 
+  // Every push into every CTA's receive buffer is visible after this barrier;
+  // afterwards no CTA touches another's shared memory, so each may exit alone.
   __syncthreads();
   cluster_arrive();
   cluster_wait();
 
   if (warp >= kEpiWarp0) {
-    // CTA `rank` reduces weight rows [rank*SL, rank*SL + SL) over all S partials.
+    // This CTA owns weight rows [rank*SL, rank*SL + SL) of the tile: sum the
+    // S slices in rank order, scale, cast and store.  Four token rows per item.
     const int SL = kBM / S;
-    const int r0 = rank * SL;
     const int t = threadIdx.x - kEpiWarp0 * 32;
-    const uint32_t part_local = smem_u32(part);
-    uint32_t base[8];
-#pragma unroll
-    for (int s = 0; s < 8; ++s) base[s] = s < S ? mapa_shared(part_local, static_cast<uint32_t>(s)) : 0u;
-    const int total = p.rows * SL;
-    for (int idx = t; idx < total; idx += 128) {
+    const int m4n = (p.rows + 3) >> 2;
+    const int items = SL * m4n;
+    for (int idx = t; idx < items; idx += 128) {
       const int nl = idx % SL;
-      const int m = idx / SL;
-      const int n = n0 + r0 + nl;
+      const int m = (idx / SL) * 4;
+      const int n = n0 + rank * SL + nl;
       if (n >= p.N) continue;
-      const uint32_t off = static_cast<uint32_t>(((r0 + nl) * L::kPitch + m) * 4);
-      float acc = 0.0f;
-      for (int s = 0; s < S; ++s) acc = __fadd_rn(acc, ld_dsmem_f32(base[s] + off));
-      const float y = __fmul_rn(__fmul_rn(acc, __ldg(p.s_x + m)), __ldg(p.s_w + n));
-      p.Y[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(y);
+      float4 acc = *reinterpret_cast<const float4*>(recv + nl * L::kPitch + m);
+      for (int s2 = 1; s2 < S; ++s2) {
+        const float4 v = *reinterpret_cast<const float4*>(recv + (s2 * SL + nl) * L::kPitch + m);
+        acc.x = __fadd_rn(acc.x, v.x);
+        acc.y = __fadd_rn(acc.y, v.y);
+        acc.z = __fadd_rn(acc.z, v.z);
+        acc.w = __fadd_rn(acc.w, v.w);
+      }
+      const float sw = __ldg(p.s_w + n);
+      const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (m + j < p.rows)
+          p.Y[static_cast<int64_t>(m + j) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(a[j], __ldg(p.s_x + m + j)), sw));
     }
   }
 
-  // No CTA may leave while the others still read its shared memory.
   __syncthreads();
-  cluster_arrive();
-  cluster_wait();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);

@@ -324,3 +324,18 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
   return r;
 }
 }  // namespace fp8q
+
+namespace fp8q {
+// 16-byte store into (possibly another CTA's) shared memory, shared::cluster address.
+__device__ __forceinline__ void st_dsmem_v4(uint32_t cluster_addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+}  // namespace fp8q
+
+namespace fp8q {
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+}  // namespace fp8q

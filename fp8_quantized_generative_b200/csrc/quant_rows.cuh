@@ -61,9 +61,11 @@ template <int TPR, int VPT>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const __half* __restrict__ X, int M, int K,
                                                         uint8_t* __restrict__ Q, float* __restrict__ S) {
   static_assert(TPR >= 32 && TPR <= 256 && (TPR & (TPR - 1)) == 0, "TPR");
-  // Let a dependent GEMM launched with programmatic serialization start its
-  // set-up now; it waits for this grid's results before reading them.
+  // Programmatic dependent launch: let the next kernel start its set-up now
+  // (it waits for this grid before touching our outputs), and wait for the
+  // previous kernel before reading X or writing Q and S.
   pdl_launch_dependents();
+  pdl_wait_prior_grid();
   constexpr int kRowsPerCta = 256 / TPR;
   constexpr int kWarpsPerRow = TPR / 32;
   __shared__ float red[8];
@@ -114,6 +116,7 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const __half* __re
                                                              uint8_t* __restrict__ Q, float* __restrict__ S) {
   __shared__ float red[8];
   pdl_launch_dependents();
+  pdl_wait_prior_grid();
   const int row = blockIdx.x;
   const int nvec = K >> 3;
   const uint4* src = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(row) * K);
@@ -146,27 +149,37 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ x, int64_t n, uint8
   }
 }
 
+// Launch on `st` with programmatic stream serialization, so that the launch
+// and prologue overlap the previous kernel on the stream.
+template <typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Host-side launcher: picks (TPR, VPT) so one row fits in registers.
 inline cudaError_t launch_quant_rows(const __half* X, int M, int K, uint8_t* Q, float* S, cudaStream_t st) {
   const int nvec = K / 8;
   int tpr = 32;
   while (tpr < 256 && tpr * 8 < nvec) tpr *= 2;
   const int vpt_needed = (nvec + tpr - 1) / tpr;
-  if (vpt_needed > 8) {
-    quant_rows_long_kernel<<<M, 256, 0, st>>>(X, M, K, Q, S);
-    return cudaGetLastError();
-  }
+  if (vpt_needed > 8) return launch_pdl(quant_rows_long_kernel, dim3(M), dim3(256), st, X, M, K, Q, S);
   const int rows_per_cta = 256 / tpr;
   const dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
   const int vpt = vpt_needed <= 1 ? 1 : vpt_needed <= 2 ? 2 : vpt_needed <= 4 ? 4 : 8;
-#define FP8Q_QR_CASE(T, V)                                                   \
-  if (tpr == T && vpt == V) {                                                \
-    quant_rows_kernel<T, V><<<grid, 256, 0, st>>>(X, M, K, Q, S);            \
-    return cudaGetLastError();                                               \
-  }
+#define FP8Q_QR_CASE(T, V) \
+  if (tpr == T && vpt == V) return launch_pdl(quant_rows_kernel<T, V>, grid, dim3(256), st, X, M, K, Q, S);
   FP8Q_QR_CASE(32, 1) FP8Q_QR_CASE(32, 2) FP8Q_QR_CASE(32, 4) FP8Q_QR_CASE(32, 8)
   FP8Q_QR_CASE(64, 8) FP8Q_QR_CASE(128, 8) FP8Q_QR_CASE(256, 8)
-  FP8Q_QR_CASE(64, 4) FP8Q_QR_CASE(128, 4) FP8Q_QR_CASE(256, 4)
 #undef FP8Q_QR_CASE
   return cudaErrorInvalidConfiguration;
 }

@@ -30,7 +30,9 @@ def run_gpu(fq, X, W):
     Xd, Wd = X.cuda(), W.cuda()
     Wq, s_w = fq.quantize_weight_per_channel(Wd)
     Xq, s_x = fq.quantize_rows_dynamic(Xd)
-    Y = fq.linear(Xq, s_x, Wq, s_w)
+    # NaN-filled output: any element the kernel fails to write fails the check
+    Y = torch.full((X.shape[0], W.shape[0]), float("nan"), dtype=torch.float16, device="cuda")
+    fq.linear(Xq, s_x, Wq, s_w, out=Y)
     torch.cuda.synchronize()
     return Y
 
@@ -124,7 +126,7 @@ def test_kernel_variants(fq, family, bn, M, N, K):
         fq.set_gemm_tuning(0, 0, 0)
 
 
-@pytest.mark.parametrize("ksplit", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("ksplit", [1, 2, 4, 8])
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (5, 264, 272), (16, 1000, 2048), (33, 520, 1040),
                                    (64, 256, 128), (100, 6144, 2048), (128, 4096, 4096)])
 def test_splitk_variants(fq, ksplit, M, N, K):

@@ -27,7 +27,8 @@ def run_gpu(fq, Xg, offsets, W):
     Wq, s_w = fq.quantize_weight_per_channel(W.cuda())
     Xq, s_x = fq.quantize_rows_dynamic(Xg.cuda())
     off = torch.from_numpy(np.asarray(offsets, dtype=np.int32)).cuda()
-    Y = fq.moe_grouped_linear(Xq, s_x, off, Wq, s_w)
+    Y = torch.full((Xg.shape[0], W.shape[1]), float("nan"), dtype=torch.float16, device="cuda")
+    fq.moe_grouped_linear(Xq, s_x, off, Wq, s_w, out=Y)
     torch.cuda.synchronize()
     return Y
 

@@ -420,6 +420,12 @@ def make_barrier(world, device):
     return barrier
 
 
+def replica_value(flops_per_step: float, steps: int, world: int, t_max_ms: float) -> float:
+    """Whole-job TFLOP/s of `world` independent replicas each running `steps`
+    steps: every rank's FLOPs over the slowest rank's time."""
+    return flops_per_step * steps * world / (t_max_ms * 1e-3) / 1e12
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     if world == 1:
         return x
@@ -475,12 +481,12 @@ def run_ours(args, world, rank, local):
         raise SystemExit(f"device error word 0x{flag:x} after the timed region")
 
     t_max_ms = max_over_ranks(total_ms, world, device)
-    value = plan.flops * args.steps * world / (t_max_ms * 1e-3) / 1e12
+    value = replica_value(plan.flops, args.steps, world, t_max_ms)
 
     e2e_steps = max(3, min(args.steps, 50))
     e2e_ms, h2d, d2h = timed_e2e(plan, tensors, e2e_steps)
     e2e_ms = max_over_ranks(e2e_ms, world, device)
-    e2e_value = plan.flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = replica_value(plan.flops, e2e_steps, world, e2e_ms)
 
     # roofline of each kernel; the dominant one (largest time share) is reported as "roofline"
     bf = plan.kernel_bytes_flops()
@@ -531,14 +537,30 @@ def run_ours(args, world, rank, local):
             "clocks": clocks}
 
 
+def csrc_hash() -> str:
+    """Hash of the kernel sources (the build whose DRAM counters are committed)."""
+    import hashlib
+    d = os.path.join(ROOT, "fp8_quantized_generative_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def load_traffic(kernel, workload):
-    """Per-launch DRAM traffic of `kernel` from the committed ncu summary, if one matches."""
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or
+    None when there is none for this workload or the kernels changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     try:
         with open(path) as f:
             t = json.load(f)
+        if t.get("csrc_sha256_16") != csrc_hash():
+            return None
         return t.get(workload, {}).get(kernel)
     except (OSError, ValueError):
         return None

@@ -491,7 +491,12 @@ def run_ours(args, world, rank, local):
     # roofline of each kernel; the dominant one (largest time share) is reported as "roofline"
     bf = plan.kernel_bytes_flops()
     hbm = float(peaks["hbm_gbs"])
-    fp8_peak = float(peaks["bf16_tflops"]) * FP8_OVER_BF16
+    # A tensor-bound kernel timed over a long back-to-back loop runs under the
+    # 1 kW power cap: compare it with the sustained GEMM figure; a short burst
+    # with the burst figure.
+    sustained = max(per_kernel_ms) * args.steps > 20.0 and "bf16_tflops_sustained" in peaks
+    bf16 = float(peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"])
+    fp8_peak = bf16 * FP8_OVER_BF16
     kern = {}
     for name, ms, (byt, fl) in zip(plan.kernels, per_kernel_ms, bf):
         t_c = fl / (fp8_peak * 1e12) if fl else 0.0
@@ -511,7 +516,9 @@ def run_ours(args, world, rank, local):
     d = kern[dom]
     roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
                 "frac": d["frac"], "traffic": traffic, "kernel": dom,
-                "peak_source": f"{peak_src} ({'fp8 = 2 x bf16 burst' if d['bound'] == 'tensor' else 'copy'})"}
+                "peak_source": (f"{peak_src} (fp8 = 2 x bf16 {'sustained' if sustained else 'burst'}; "
+                                f"timed loop {max(per_kernel_ms) * args.steps:.1f} ms)" if d["bound"] == "tensor"
+                                else f"{peak_src} (HBM copy)")}
     step_flops = plan.flops
     step_bytes = sum(b for b, _ in bf)
     ms_step = t_max_ms / args.steps
@@ -569,7 +576,7 @@ def load_traffic(kernel, workload):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="qkv")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

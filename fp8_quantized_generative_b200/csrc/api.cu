@@ -256,39 +256,72 @@ int max_pair_clusters(int dev) {
   return n;
 }
 
+// Tail split of the pair schedule: with F full tiles on C clusters, the
+// last F mod C tiles are cut into q in {2, 4} pieces along N when that still
+// fits one round (pieces stay multiples of 64 columns); q = 1 otherwise.
+struct TailSplit {
+  int main_tiles;
+  int q;
+};
+TailSplit tail_split(int64_t full_tiles, int clusters, int bn) {
+  // A wide tile (bn = 512) splits only into 256-column halves.
+  const int qmax = bn > 256 ? 2 : 4;
+  TailSplit r{static_cast<int>(full_tiles), 1};
+  static const bool enabled = [] {
+    const char* e = std::getenv("FP8Q_TAIL");   // tuning knob: 0 disables the split
+    return !(e && e[0] == '0');
+  }();
+  const int64_t left = full_tiles % clusters;
+  if (left == 0 || !enabled) return r;
+  for (int q = qmax; q >= 2; q >>= 1) {
+    if ((bn / q) % 64 != 0) continue;
+    if (left * q <= clusters) {
+      r.main_tiles = static_cast<int>(full_tiles - left);
+      r.q = q;
+      return r;
+    }
+  }
+  return r;
+}
+
 template <int BN, int STAGES>
-fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, const GemmParams& p, int dev, cudaStream_t st) {
+fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, const GemmParams& p0, int dev, cudaStream_t st) {
   using L = PairLayout<BN, STAGES>;
-  CUtensorMap ta, tb;
-  fp8q_status s = make_operand_map(&ta, A, p.rows, p.K, kBM);
-  if (s != FP8Q_OK) return s;
-  s = make_operand_map(&tb, B, p.N, p.K, L::kBRows);
-  if (s != FP8Q_OK) return s;
-  CUtensorMap ty;
-  s = make_output_map(&ty, p.Y, p.rows, p.N);
-  if (s != FP8Q_OK) return s;
-  auto kernel = fp8_gemm_pair_kernel<BN, STAGES>;
-  cudaError_t e = ensure_smem<fp8_gemm_pair_kernel<BN, STAGES>>(L::kSmemBytes, dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair)");
   const int clusters = max_pair_clusters<BN, STAGES>(dev);
   if (clusters < 1) {
     g_last_error = "no 2-CTA cluster of the pair GEMM fits on this device";
     return FP8Q_ERR_UNSUPPORTED;
   }
-  const int64_t tiles = int64_t((p.rows + 2 * kBM - 1) / (2 * kBM)) * ((p.N + BN - 1) / BN);
+  GemmParams p = p0;
+  const int64_t full = int64_t((p.rows + 2 * kBM - 1) / (2 * kBM)) * ((p.N + BN - 1) / BN);
+  const TailSplit ts = tail_split(full, clusters, BN);
+  p.main_tiles = ts.main_tiles;
+  p.tail_q = ts.q;
+  CUtensorMap ta, tb, tbt, ty;
+  fp8q_status s = make_operand_map(&ta, A, p.rows, p.K, kBM);
+  if (s != FP8Q_OK) return s;
+  s = make_operand_map(&tb, B, p.N, p.K, L::kWide ? 128 : L::kBRows);
+  if (s != FP8Q_OK) return s;
+  s = make_operand_map(&tbt, B, p.N, p.K, L::kWide ? 128 : L::kBRows / ts.q);
+  if (s != FP8Q_OK) return s;
+  s = make_output_map(&ty, p.Y, p.rows, p.N);
+  if (s != FP8Q_OK) return s;
+  auto kernel = fp8_gemm_pair_kernel<BN, STAGES>;
+  cudaError_t e = ensure_smem<fp8_gemm_pair_kernel<BN, STAGES>>(L::kSmemBytes, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair)");
+  const int64_t tiles = int64_t(ts.main_tiles) + (full - ts.main_tiles) * ts.q;
   const int pairs = static_cast<int>(tiles < clusters ? tiles : clusters);
-  e = launch_ex(kernel, dim3(2 * pairs), dim3(kGemmThreads), L::kSmemBytes, st, 2, true, ta, tb, ty, p);
+  e = launch_ex(kernel, dim3(2 * pairs), dim3(kGemmThreads), L::kSmemBytes, st, 2, true, ta, tb, tbt, ty, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_pair_kernel launch");
   return FP8Q_OK;
 }
 
 // Pair-kernel tile width: the candidate with the least modelled time =
-// waves of tiles x per-tile work / relative efficiency.  Narrower tiles move
-// more operand bytes out of L2 per FLOP (256 FLOP/B per SM at BN = 256,
-// 219 at 192, 171 at 128) and pay the per-tile epilogue more often; the
-// efficiency factors are per-FLOP throughputs relative to BN = 256 measured
-// on B200 (4096 x 6144 x 2048).  A narrower tile only wins when it removes a
-// mostly idle wave.
+// rounds of tiles (after the tail split) x per-tile work / relative
+// efficiency.  Narrower tiles move more operand bytes out of L2 per FLOP
+// (256 FLOP/B per SM at BN = 256, 219 at 192, 171 at 128) and pay the
+// per-tile epilogue more often; the efficiency factors are per-FLOP
+// throughputs relative to BN = 256 measured on B200 (4096 x 6144 x 2048).
 int choose_pair_bn(int64_t M, int64_t N, int clusters) {
   const int cands[3] = {256, 192, 128};
   const double eff[3] = {1.0, 0.79, 0.60};
@@ -296,9 +329,13 @@ int choose_pair_bn(int64_t M, int64_t N, int clusters) {
   double best_cost = 1e300;
   for (int i = 0; i < 3; ++i) {
     const int bn = cands[i];
-    const int64_t tiles = ((M + 255) / 256) * ((N + bn - 1) / bn);
-    const int64_t waves = (tiles + clusters - 1) / clusters;
-    const double cost = static_cast<double>(waves) * bn / eff[i];
+    const int64_t full = ((M + 255) / 256) * ((N + bn - 1) / bn);
+    const TailSplit ts = tail_split(full, clusters, bn);
+    const int64_t rounds_main = ts.main_tiles / clusters;
+    const int64_t rest = (full - ts.main_tiles) * ts.q;   // pieces after the full rounds
+    const double rounds = static_cast<double>(rounds_main + (ts.main_tiles % clusters ? 1 : 0)) +
+                          static_cast<double>((rest + clusters - 1) / clusters) / ts.q;
+    const double cost = rounds * bn / eff[i];
     if (cost < best_cost * 0.999) {
       best_cost = cost;
       best = bn;
@@ -346,11 +383,13 @@ int max_splitk_clusters(int dev, int S) {
 // Split factor S in {1, 2, 4, 8} (a divisor of the 128 weight rows of a
 // tile, so each CTA of the cluster owns an equal slice of the reduction):
 // the largest that keeps every cluster of the grid resident at once (one
-// wave) and gives each CTA at least one K block.
+// wave; two CTAs share an SM when their shared memory allows) and gives
+// each CTA at least one K block.
 template <int MPAD, int STAGES>
 int choose_ksplit(int dev, int sms, int n_tiles, int num_kb) {
+  (void)sms;
   int S = 8;
-  while (S > 1 && (n_tiles * S > sms || S > num_kb)) S >>= 1;
+  while (S > 1 && S > num_kb) S >>= 1;
   while (S > 1) {
     const int fit = max_splitk_clusters<MPAD, STAGES>(dev, S);
     if (fit >= n_tiles) break;
@@ -406,6 +445,7 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
     switch (bn) {
       case 128: return launch_pair<128, 8>(Xq, Wq, q, dev, st);
       case 192: return launch_pair<192, 7>(Xq, Wq, q, dev, st);
+      case 512: return launch_pair<512, 4>(Xq, Wq, q, dev, st);
       default: return launch_pair<256, 6>(Xq, Wq, q, dev, st);
     }
   }
@@ -484,6 +524,8 @@ fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, 
   p.K = static_cast<int>(K);
   p.E = 1;
   p.n_fastest = 0;
+  p.main_tiles = 0;
+  p.tail_q = 1;
   return launch_dense(Xq, Wq, p, static_cast<cudaStream_t>(stream));
 }
 
@@ -508,6 +550,8 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const i
   p.K = static_cast<int>(K);
   p.E = E;
   p.n_fastest = 0;
+  p.main_tiles = 0;
+  p.tail_q = 1;
   const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBNGrouped - 1) / kBNGrouped);
   return launch_gemm<true>(Xq, rows, Wq, int64_t(E) * N, p, tiles, static_cast<cudaStream_t>(stream));
 }
@@ -530,7 +574,8 @@ fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* 
 
 fp8q_status fp8q_set_gemm_tuning(int kernel_family, int tile_n, int ksplit) {
   if (kernel_family < 0 || kernel_family > 3) return invalid("kernel_family must be 0, 1, 2 or 3");
-  if (tile_n != 0 && tile_n != 128 && tile_n != 192 && tile_n != 256) return invalid("tile_n must be 0, 128, 192 or 256");
+  if (tile_n != 0 && tile_n != 128 && tile_n != 192 && tile_n != 256 && tile_n != 512)
+    return invalid("tile_n must be 0, 128, 192, 256 or 512");
   if (ksplit != 0 && ksplit != 1 && ksplit != 2 && ksplit != 4 && ksplit != 8)
     return invalid("ksplit must be 0, 1, 2, 4 or 8");
   knobs().force = kernel_family;

@@ -34,6 +34,11 @@ struct GemmParams {
   int K;
   int E;                    // 1 for dense
   int n_fastest;            // dense tile order: 1 = walk n-blocks first
+  // CTA-pair kernel tail split: the first main_tiles full tiles run at full
+  // width; each remaining full tile is cut along N into tail_q pieces
+  // (tail_q in {1, 2, 4}) so that the last round keeps every cluster busy.
+  int main_tiles;
+  int tail_q;
 };
 
 // One output slab of a CTA: 128 rows starting at row0, BN columns at n0.
@@ -59,19 +64,18 @@ __device__ __forceinline__ uint32_t stage_off(int r, int c) {
 // 32 columns at a time: TMEM -> registers -> scale and cast -> swizzled
 // staging tile in shared memory -> one bulk tensor store (or, for a slab cut
 // by an expert boundary, coalesced row-masked stores).
-template <int BN>
+// `bn` is the slab width (a multiple of 64; each warp takes bn/2 columns).
 __device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams& p, const CUtensorMap* tmY,
-                                              uint32_t tmem_acc, int warp, int lane, uint8_t* stage) {
-  static_assert(BN % 64 == 0, "each epilogue warp takes BN/2 columns in chunks of 32");
+                                              uint32_t tmem_acc, int warp, int lane, uint8_t* stage, int bn) {
   const int q = warp & 3;
   const int h = (warp - kEpiWarp0) >> 2;
   const int r = t.row0 + q * 32 + lane;
   const float sx = r < t.row_end ? __ldg(p.s_x + r) : 0.0f;
   const uint32_t sbase = smem_u32(stage);
-  const uint32_t taddr0 = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * (BN / 2));
+  const uint32_t taddr0 = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * (bn / 2));
 #pragma unroll 1
-  for (int j = 0; j < BN / 64; ++j) {
-    const int cl = h * (BN / 2) + j * 32;   // first column of the chunk within the tile
+  for (int j = 0; j < bn / 64; ++j) {
+    const int cl = h * (bn / 2) + j * 32;   // first column of the chunk within the tile
     const int colw = t.n0 + cl + lane;
     const float sw_lane = colw < p.N ? __ldg(p.s_w + t.sw0 + cl + lane) : 0.0f;
     uint32_t v[32];

@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // A bulk store clips only at the tensor edge, so it is used unless the
       // slab crosses into the next expert's rows.
       et.tma = !kGrouped || c.a_row0 + kBM <= c.row_end;
-      epilogue_slab<BN>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage);
+      epilogue_slab(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);

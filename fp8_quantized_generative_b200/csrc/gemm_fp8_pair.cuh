@@ -15,6 +15,10 @@
 //   * each CTA's eight epilogue warps drain their own 128 TMEM lanes
 //     (gemm_common.cuh: bulk tensor stores through a swizzled staging tile)
 //     and arrive on the leader's "accumulator empty" barrier.
+// When the full tiles do not divide evenly over the clusters, the leftover
+// tiles are cut along N into 2 or 4 narrower pieces (a runtime MMA N and a
+// second B descriptor with a narrower box), so the last round is short
+// instead of mostly idle.
 // No TMA multicast: every CTA loads only the tiles it stores.
 #pragma once
 
@@ -30,17 +34,52 @@ struct PairLayout {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kNumBars = 2 * STAGES + 5;      // full, empty, tfull[2], tempty[2], drain
   static constexpr int kTmemCols = 512;
+  // BN <= 256: two TMEM accumulators (the epilogue of one tile overlaps the
+  // MMAs of the next).  BN = 512 ("wide"): one accumulator filling TMEM,
+  // computed as two N = 256 halves per k-step; a third less operand traffic
+  // per FLOP, but the epilogue no longer overlaps the next tile's MMAs.
+  static constexpr bool kWide = BN > 256;
+  static constexpr int kNAcc = kWide ? 1 : 2;
   static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes + kEpiSmemBytes + kNumBars * 8 + 32;
 };
+
+// Tile t of the pair schedule: full tiles first, then the tail pieces.
+struct PairTile {
+  int m_blk;
+  int n0;      // first output column
+  int bn;      // width: BN, or BN / tail_q for a tail piece
+  bool tail;
+};
+
+template <int BN>
+__device__ __forceinline__ PairTile pair_tile(int t, const GemmParams& p, int num_m, int num_n) {
+  PairTile r;
+  int f, piece = 0;
+  r.tail = t >= p.main_tiles;
+  if (!r.tail) {
+    f = t;
+  } else {
+    const int u = t - p.main_tiles;
+    f = p.main_tiles + u / p.tail_q;
+    piece = u % p.tail_q;
+  }
+  const int n_blk = p.n_fastest ? f % num_n : f / num_m;
+  r.m_blk = p.n_fastest ? f / num_n : f % num_m;
+  r.bn = r.tail ? BN / p.tail_q : BN;
+  r.n0 = n_blk * BN + piece * r.bn;
+  return r;
+}
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+                         const __grid_constant__ CUtensorMap tmBt, const __grid_constant__ CUtensorMap tmY,
+                         const GemmParams p) {
   using L = PairLayout<BN, STAGES>;
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256 && (BN / 2) % 8 == 0, "BN");
-  static_assert(2 * BN <= L::kTmemCols, "two accumulators must fit in TMEM");
-  constexpr uint32_t kIdesc = idesc_e4m3_f32(2 * kBM, BN);
+  static_assert(BN % 64 == 0 && BN >= 64 && (BN <= 256 || BN == 512) && (BN / 2) % 8 == 0, "BN");
+  static_assert(L::kNAcc * BN <= L::kTmemCols, "accumulators must fit in TMEM");
+  constexpr bool kWide = L::kWide;
+  constexpr uint32_t kIdesc = idesc_e4m3_f32(2 * kBM, kWide ? 256 : BN);
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -66,7 +105,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int num_m = (p.rows + 2 * kBM - 1) / (2 * kBM);
   const int num_n = (p.N + BN - 1) / BN;
   const int num_kb = (p.K + kBK - 1) / kBK;
-  const int total = num_m * num_n;
+  const int total = p.main_tiles + (num_m * num_n - p.main_tiles) * p.tail_q;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -84,6 +123,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmBt);
     prefetch_tmap(&tmY);
   }
   if (warp == 1) {
@@ -103,6 +143,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
+    // This CTA's share of a tile's weight rows for one k-block.  Normal
+    // tiles: rows n0 + rank*bn/2 .. +bn/2.  Wide tiles: for each 256-column
+    // half h, rows n0 + 256h + rank*128 .. +128, stored one after the other.
+    auto load_b = [&](const PairTile& pt, uint8_t* dst, uint32_t bar, int kx) {
+      if (kWide) {
+        for (int h = 0; h < pt.bn / 256; ++h)
+          tma_load_2d_pair(dst + h * 128 * kBK, &tmB, bar, kx, pt.n0 + 256 * h + static_cast<int>(rank) * 128);
+      } else {
+        tma_load_2d_pair(dst, pt.tail ? &tmBt : &tmB, bar, kx, pt.n0 + static_cast<int>(rank) * (pt.bn / 2));
+      }
+    };
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
@@ -113,21 +164,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // tiles wait.
       int pre = 0;
       if (pair < total) {
-        const int n_blk = p.n_fastest ? pair % num_n : pair / num_m;
-        const int b_row = n_blk * BN + static_cast<int>(rank) * L::kBRows;
+        const PairTile pt = pair_tile<BN>(pair, p, num_m, num_n);
+        const uint32_t bytes = 2u * static_cast<uint32_t>(L::kABytes + (pt.bn / 2) * kBK);
         pre = num_kb < STAGES ? num_kb : STAGES;
         for (int i = 0; i < pre; ++i) {
           const uint32_t full_leader = mapa_shared(smem_u32(&full[i]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[i], 2 * L::kStageBytes);
-          tma_load_2d_pair(sB + i * L::kBBytes, &tmB, full_leader, i * kBK, b_row);
+          if (leader) mbar_arrive_expect_tx(&full[i], bytes);
+          load_b(pt, sB + i * L::kBBytes, full_leader, i * kBK);
         }
       }
       pdl_wait_prior_grid();
       for (int t = pair; t < total && ok; t += npairs) {
-        const int m_blk = p.n_fastest ? t / num_n : t % num_m;
-        const int n_blk = p.n_fastest ? t % num_n : t / num_m;
-        const int a_row = m_blk * 2 * kBM + static_cast<int>(rank) * kBM;
-        const int b_row = n_blk * BN + static_cast<int>(rank) * L::kBRows;
+        const PairTile pt = pair_tile<BN>(t, p, num_m, num_n);
+        const int a_row = pt.m_blk * 2 * kBM + static_cast<int>(rank) * kBM;
+        const uint32_t bytes = 2u * static_cast<uint32_t>(L::kABytes + (pt.bn / 2) * kBK);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (pre > 0) {
             // stage kb of the first pass: weights already requested
@@ -145,9 +195,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           const uint32_t full_leader = mapa_shared(smem_u32(&full[s]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[s], 2 * L::kStageBytes);
+          if (leader) mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d_pair(sA + s * L::kABytes, &tmA, full_leader, kb * kBK, a_row);
-          tma_load_2d_pair(sB + s * L::kBBytes, &tmB, full_leader, kb * kBK, b_row);
+          load_b(pt, sB + s * L::kBBytes, full_leader, kb * kBK);
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;
@@ -179,6 +229,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t idesc = (!kWide && t >= p.main_tiles) ? idesc_e4m3_f32(2 * kBM, BN / p.tail_q) : kIdesc;
+        const int halves = kWide ? pair_tile<BN>(t, p, num_m, num_n).bn / 256 : 1;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {
             ok = false;
@@ -189,8 +241,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t b0 = sw128_kmajor_desc(smem_u32(sB + s * L::kBBytes));
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k)
-            mma_f8f6f4_pair(d, a0 + static_cast<uint64_t>(k * kUmmaK / 16),
-                            b0 + static_cast<uint64_t>(k * kUmmaK / 16), kIdesc, (kb | k) != 0 ? 1u : 0u);
+            for (int h = 0; h < halves; ++h)   // wide: N = 256 halves at TMEM columns 256h
+              mma_f8f6f4_pair(d + static_cast<uint32_t>(256 * h), a0 + static_cast<uint64_t>(k * kUmmaK / 16),
+                              b0 + static_cast<uint64_t>(h * 128 * kBK / 16 + k * kUmmaK / 16), idesc,
+                              (kb | k) != 0 ? 1u : 0u);
           issued = true;
           mma_commit_pair_mc(&empty[s], 0x3);
           if (++s == STAGES) {
@@ -200,8 +254,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         mma_commit_pair_mc(&tfull[acc], 0x3);
-        acc ^= 1;
-        if (acc == 0) acc_ph ^= 1u;
+        if (++acc == L::kNAcc) {
+          acc = 0;
+          acc_ph ^= 1u;
+        }
       }
       if (!ok) {
         raise_error(0x2u);
@@ -222,8 +278,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int t = pair; t < total; t += npairs) {
-      const int m_blk = p.n_fastest ? t / num_n : t % num_m;
-      const int n_blk = p.n_fastest ? t % num_n : t / num_m;
+      const PairTile pt = pair_tile<BN>(t, p, num_m, num_n);
       if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
         raise_error(0x4u);
         *abort_flag = 1;
@@ -231,17 +286,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       EpiTile et;
-      et.row0 = m_blk * 2 * kBM + static_cast<int>(rank) * kBM;
+      et.row0 = pt.m_blk * 2 * kBM + static_cast<int>(rank) * kBM;
       et.row_end = p.rows;
-      et.n0 = n_blk * BN;
+      et.n0 = pt.n0;
       et.sw0 = et.n0;
       et.tma = true;   // dense: the bulk store clips at the tensor edge
-      epilogue_slab<BN>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage);
+      epilogue_slab(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, pt.bn);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-      acc ^= 1;
-      if (acc == 0) acc_ph ^= 1u;
+      if (++acc == L::kNAcc) {
+        acc = 0;
+        acc_ph ^= 1u;
+      }
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();

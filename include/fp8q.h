@@ -144,7 +144,7 @@ fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* 
  * single-CTA kernel (128-row tiles), 2 = the CTA-pair kernel (256-row tiles,
  * tcgen05 cta_group::2), 3 = the swap-AB split-K cluster kernel (M <= 128
  * only; larger M falls back to automatic).  tile_n: 0 = automatic, else 128,
- * 192 or 256 (pair kernel only).  ksplit: 0 = automatic, else the split-K
+ * 192, 256 or 512 (pair kernel only).  ksplit: 0 = automatic, else the split-K
  * cluster size 1, 2, 4 or 8 (split-K kernel only).  Process-wide; not thread-safe against
  * concurrent launches.  Environment variables FP8Q_FORCE_KERNEL
  * (auto|single|pair|splitk), FP8Q_BN and FP8Q_KSPLIT (split-K cluster size,

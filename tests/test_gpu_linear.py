@@ -111,7 +111,7 @@ def test_zero_rows_noop(fq):
     assert Y.shape == (0, 64)
 
 
-VARIANTS = [(1, 0), (2, 128), (2, 192), (2, 256)]
+VARIANTS = [(1, 0), (2, 128), (2, 192), (2, 256), (2, 512)]
 
 
 @pytest.mark.parametrize("family,bn", VARIANTS)

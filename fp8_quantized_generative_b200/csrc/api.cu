@@ -224,22 +224,23 @@ fp8q_status launch_gemm(const uint8_t* A, int64_t a_rows, const uint8_t* B, int6
 }
 
 // Per-device cache of how many 2-CTA clusters of a pair kernel fit at once.
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool kGrouped>
 int max_pair_clusters(int dev) {
   static int cache[kMaxDevices] = {0};
   static std::mutex mu;
   std::lock_guard<std::mutex> g(mu);
   if (cache[dev] > 0) return cache[dev];
   using L = PairLayout<BN, STAGES>;
-  auto kernel = fp8_gemm_pair_kernel<BN, STAGES>;
-  if (ensure_smem<fp8_gemm_pair_kernel<BN, STAGES>>(L::kSmemBytes, dev) != cudaSuccess) {
+  auto kernel = fp8_gemm_pair_kernel<BN, STAGES, kGrouped>;
+  const size_t smem = L::smem_bytes(kGrouped ? kMaxExperts : 0);
+  if (ensure_smem<fp8_gemm_pair_kernel<BN, STAGES, kGrouped>>(smem, dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return 0;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2);
   cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = L::kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
   attr.val.clusterDim.x = 2;
@@ -284,34 +285,48 @@ TailSplit tail_split(int64_t full_tiles, int clusters, int bn) {
   return r;
 }
 
-template <int BN, int STAGES>
-fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, const GemmParams& p0, int dev, cudaStream_t st) {
+// Launch a pair kernel.  Dense: A = Xq [rows, K], B = Wq [N, K].  Grouped:
+// B = Wq [E*N, K] and the schedule comes from the device offsets;
+// `tiles_upper_bound` caps the grid when the tile count is unknown on the host.
+template <int BN, int STAGES, bool kGrouped>
+fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, int64_t b_rows, const GemmParams& p0, int dev,
+                        cudaStream_t st, int64_t tiles_upper_bound = 0) {
   using L = PairLayout<BN, STAGES>;
-  const int clusters = max_pair_clusters<BN, STAGES>(dev);
+  const int clusters = max_pair_clusters<BN, STAGES, kGrouped>(dev);
   if (clusters < 1) {
     g_last_error = "no 2-CTA cluster of the pair GEMM fits on this device";
     return FP8Q_ERR_UNSUPPORTED;
   }
   GemmParams p = p0;
-  const int64_t full = int64_t((p.rows + 2 * kBM - 1) / (2 * kBM)) * ((p.N + BN - 1) / BN);
-  const TailSplit ts = tail_split(full, clusters, BN);
-  p.main_tiles = ts.main_tiles;
-  p.tail_q = ts.q;
+  int64_t tiles;
+  TailSplit ts{0, 1};
+  if (kGrouped) {
+    p.main_tiles = 0;
+    p.tail_q = 1;
+    tiles = tiles_upper_bound;
+  } else {
+    const int64_t full = int64_t((p.rows + 2 * kBM - 1) / (2 * kBM)) * ((p.N + BN - 1) / BN);
+    ts = tail_split(full, clusters, BN);
+    p.main_tiles = ts.main_tiles;
+    p.tail_q = ts.q;
+    tiles = int64_t(ts.main_tiles) + (full - ts.main_tiles) * ts.q;
+  }
   CUtensorMap ta, tb, tbt, ty;
   fp8q_status s = make_operand_map(&ta, A, p.rows, p.K, kBM);
   if (s != FP8Q_OK) return s;
-  s = make_operand_map(&tb, B, p.N, p.K, L::kWide ? 128 : L::kBRows);
+  s = make_operand_map(&tb, B, b_rows, p.K, L::kWide ? 128 : L::kBRows);
   if (s != FP8Q_OK) return s;
-  s = make_operand_map(&tbt, B, p.N, p.K, L::kWide ? 128 : L::kBRows / ts.q);
+  s = make_operand_map(&tbt, B, b_rows, p.K, L::kWide ? 128 : L::kBRows / ts.q);
   if (s != FP8Q_OK) return s;
   s = make_output_map(&ty, p.Y, p.rows, p.N);
   if (s != FP8Q_OK) return s;
-  auto kernel = fp8_gemm_pair_kernel<BN, STAGES>;
-  cudaError_t e = ensure_smem<fp8_gemm_pair_kernel<BN, STAGES>>(L::kSmemBytes, dev);
+  auto kernel = fp8_gemm_pair_kernel<BN, STAGES, kGrouped>;
+  cudaError_t e = ensure_smem<fp8_gemm_pair_kernel<BN, STAGES, kGrouped>>(
+      L::smem_bytes(kGrouped ? kMaxExperts : 0), dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair)");
-  const int64_t tiles = int64_t(ts.main_tiles) + (full - ts.main_tiles) * ts.q;
-  const int pairs = static_cast<int>(tiles < clusters ? tiles : clusters);
-  e = launch_ex(kernel, dim3(2 * pairs), dim3(kGemmThreads), L::kSmemBytes, st, 2, true, ta, tb, tbt, ty, p);
+  const int pairs = static_cast<int>(tiles < clusters ? (tiles < 1 ? 1 : tiles) : clusters);
+  e = launch_ex(kernel, dim3(2 * pairs), dim3(kGemmThreads), L::smem_bytes(kGrouped ? p.E : 0), st, 2, true, ta, tb,
+                tbt, ty, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_pair_kernel launch");
   return FP8Q_OK;
 }
@@ -440,13 +455,13 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
   if (kn.force == 1) pair = false;
   if (kn.force == 2) pair = true;
   if (pair) {
-    const int clusters = max_pair_clusters<256, 6>(dev);
+    const int clusters = max_pair_clusters<256, 6, false>(dev);
     int bn = kn.bn ? kn.bn : choose_pair_bn(p.rows, p.N, clusters > 0 ? clusters : sms / 2);
     switch (bn) {
-      case 128: return launch_pair<128, 8>(Xq, Wq, q, dev, st);
-      case 192: return launch_pair<192, 7>(Xq, Wq, q, dev, st);
-      case 512: return launch_pair<512, 4>(Xq, Wq, q, dev, st);
-      default: return launch_pair<256, 6>(Xq, Wq, q, dev, st);
+      case 128: return launch_pair<128, 8, false>(Xq, Wq, p.N, q, dev, st);
+      case 192: return launch_pair<192, 7, false>(Xq, Wq, p.N, q, dev, st);
+      case 512: return launch_pair<512, 4, false>(Xq, Wq, p.N, q, dev, st);
+      default: return launch_pair<256, 6, false>(Xq, Wq, p.N, q, dev, st);
     }
   }
   const int64_t tiles = int64_t((p.rows + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
@@ -552,6 +567,17 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const i
   p.n_fastest = 0;
   p.main_tiles = 0;
   p.tail_q = 1;
+  // Single-CTA 128-row tiles by default; kernel family 2 selects CTA-pair
+  // tiles of 256 expert rows (each weight tile read by half as many row
+  // blocks), which measured no faster for the up projection and slower for
+  // the down projection (8 K blocks per tile) on B200.
+  if (knobs().force == 2) {
+    int dev = 0, sms = 0;
+    const cudaError_t e = current_device_info(&dev, &sms);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    const int64_t tiles = ((rows + 2 * kBM - 1) / (2 * kBM) + E) * ((N + 255) / 256);
+    return launch_pair<256, 6, true>(Xq, Wq, int64_t(E) * N, p, dev, static_cast<cudaStream_t>(stream), tiles);
+  }
   const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBNGrouped - 1) / kBNGrouped);
   return launch_gemm<true>(Xq, rows, Wq, int64_t(E) * N, p, tiles, static_cast<cudaStream_t>(stream));
 }

@@ -41,19 +41,47 @@ struct PairLayout {
   static constexpr bool kWide = BN > 256;
   static constexpr int kNAcc = kWide ? 1 : 2;
   static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes + kEpiSmemBytes + kNumBars * 8 + 32;
+  // plus the MoE schedule tables (offsets and tile prefix) when grouped
+  static size_t smem_bytes(int E) { return kSmemBytes + 2 * static_cast<size_t>(E + 1) * 4 + 16; }
 };
 
-// Tile t of the pair schedule: full tiles first, then the tail pieces.
+// Tile t of the pair schedule.  Dense: full tiles first, then the tail
+// pieces.  Grouped (MoE): tiles ordered (expert, n-block, 256-row block) from
+// the device-side tile prefix, so the row blocks sharing an expert's weight
+// tile run back to back.
 struct PairTile {
-  int m_blk;
-  int n0;      // first output column
-  int bn;      // width: BN, or BN / tail_q for a tail piece
+  int a_row0;   // first of the pair's 256 token rows
+  int row_end;  // rows >= row_end are not stored (end of matrix or expert group)
+  int b_row0;   // first weight row of the tile
+  int n0;       // first output column
+  int sw0;      // s_w index of column n0
+  int bn;       // width: BN, or BN / tail_q for a tail piece
   bool tail;
 };
 
-template <int BN>
-__device__ __forceinline__ PairTile pair_tile(int t, const GemmParams& p, int num_m, int num_n) {
+template <int BN, bool kGrouped>
+__device__ __forceinline__ PairTile pair_tile(int t, const GemmParams& p, int num_m, int num_n,
+                                              const int* tile_prefix, const int* offs) {
   PairTile r;
+  if (kGrouped) {
+    int lo = 0, hi = p.E;   // tile_prefix[lo] <= t < tile_prefix[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tile_prefix[mid] <= t) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int mt = (offs[e + 1] - offs[e] + 2 * kBM - 1) / (2 * kBM);
+    const int local = t - tile_prefix[e];
+    const int n_blk = local / mt;
+    r.a_row0 = offs[e] + (local - n_blk * mt) * 2 * kBM;
+    r.row_end = offs[e + 1];
+    r.n0 = n_blk * BN;
+    r.b_row0 = e * p.N + r.n0;
+    r.sw0 = r.b_row0;
+    r.bn = BN;
+    r.tail = false;
+    return r;
+  }
   int f, piece = 0;
   r.tail = t >= p.main_tiles;
   if (!r.tail) {
@@ -64,13 +92,17 @@ __device__ __forceinline__ PairTile pair_tile(int t, const GemmParams& p, int nu
     piece = u % p.tail_q;
   }
   const int n_blk = p.n_fastest ? f % num_n : f / num_m;
-  r.m_blk = p.n_fastest ? f / num_n : f % num_m;
+  const int m_blk = p.n_fastest ? f / num_n : f % num_m;
   r.bn = r.tail ? BN / p.tail_q : BN;
   r.n0 = n_blk * BN + piece * r.bn;
+  r.a_row0 = m_blk * 2 * kBM;
+  r.row_end = p.rows;
+  r.b_row0 = r.n0;
+  r.sw0 = r.n0;
   return r;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool kGrouped>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmBt, const __grid_constant__ CUtensorMap tmY,
@@ -95,6 +127,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = bars + 2 * STAGES + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* total_s = reinterpret_cast<int*>(tmem_slot + 2);
+  int* tile_prefix = reinterpret_cast<int*>(tmem_slot + 8);
+  int* offs = tile_prefix + (p.E + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -105,7 +140,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int num_m = (p.rows + 2 * kBM - 1) / (2 * kBM);
   const int num_n = (p.N + BN - 1) / BN;
   const int num_kb = (p.K + kBK - 1) / kBK;
-  const int total = p.main_tiles + (num_m * num_n - p.main_tiles) * p.tail_q;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -137,6 +171,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cluster_arrive();
   cluster_wait();
   const uint32_t tmem_base = *tmem_slot;
+  int total;
+  if (kGrouped) {
+    // The expert offsets may come from the previous kernel: wait for it, then
+    // build the tile schedule (and check the offsets) on the device.
+    pdl_wait_prior_grid();
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) offs[i] = __ldg(p.offsets + i);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      bool ok = offs[0] == 0 && offs[p.E] == p.rows;
+      int acc = 0;
+      for (int e = 0; e < p.E; ++e) {
+        const int cnt = offs[e + 1] - offs[e];
+        ok = ok && cnt >= 0;
+        tile_prefix[e] = acc;
+        acc += (cnt > 0 ? (cnt + 2 * kBM - 1) / (2 * kBM) : 0) * num_n;
+      }
+      tile_prefix[p.E] = acc;
+      *total_s = ok ? acc : 0;
+      if (!ok && blockIdx.x == 0) raise_error(0x8u);
+    }
+    __syncthreads();
+    total = *total_s;
+  } else {
+    total = p.main_tiles + (num_m * num_n - p.main_tiles) * p.tail_q;
+  }
   // The next kernel on the stream may begin launching (it waits for this
   // grid before touching anything this grid reads or writes).
   pdl_launch_dependents();
@@ -149,9 +208,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto load_b = [&](const PairTile& pt, uint8_t* dst, uint32_t bar, int kx) {
       if (kWide) {
         for (int h = 0; h < pt.bn / 256; ++h)
-          tma_load_2d_pair(dst + h * 128 * kBK, &tmB, bar, kx, pt.n0 + 256 * h + static_cast<int>(rank) * 128);
+          tma_load_2d_pair(dst + h * 128 * kBK, &tmB, bar, kx, pt.b_row0 + 256 * h + static_cast<int>(rank) * 128);
       } else {
-        tma_load_2d_pair(dst, pt.tail ? &tmBt : &tmB, bar, kx, pt.n0 + static_cast<int>(rank) * (pt.bn / 2));
+        tma_load_2d_pair(dst, pt.tail ? &tmBt : &tmB, bar, kx, pt.b_row0 + static_cast<int>(rank) * (pt.bn / 2));
       }
     };
     if (lane == 0) {
@@ -163,8 +222,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // first tile's weight tiles before waiting for it; only the activation
       // tiles wait.
       int pre = 0;
-      if (pair < total) {
-        const PairTile pt = pair_tile<BN>(pair, p, num_m, num_n);
+      if (!kGrouped && pair < total) {
+        const PairTile pt = pair_tile<BN, kGrouped>(pair, p, num_m, num_n, tile_prefix, offs);
         const uint32_t bytes = 2u * static_cast<uint32_t>(L::kABytes + (pt.bn / 2) * kBK);
         pre = num_kb < STAGES ? num_kb : STAGES;
         for (int i = 0; i < pre; ++i) {
@@ -175,8 +234,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       pdl_wait_prior_grid();
       for (int t = pair; t < total && ok; t += npairs) {
-        const PairTile pt = pair_tile<BN>(t, p, num_m, num_n);
-        const int a_row = pt.m_blk * 2 * kBM + static_cast<int>(rank) * kBM;
+        const PairTile pt = pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs);
+        const int a_row = pt.a_row0 + static_cast<int>(rank) * kBM;
         const uint32_t bytes = 2u * static_cast<uint32_t>(L::kABytes + (pt.bn / 2) * kBK);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (pre > 0) {
@@ -230,7 +289,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
         const uint32_t idesc = (!kWide && t >= p.main_tiles) ? idesc_e4m3_f32(2 * kBM, BN / p.tail_q) : kIdesc;
-        const int halves = kWide ? pair_tile<BN>(t, p, num_m, num_n).bn / 256 : 1;
+        const int halves = kWide ? pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs).bn / 256 : 1;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {
             ok = false;
@@ -278,7 +337,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int t = pair; t < total; t += npairs) {
-      const PairTile pt = pair_tile<BN>(t, p, num_m, num_n);
+      const PairTile pt = pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs);
       if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
         raise_error(0x4u);
         *abort_flag = 1;
@@ -286,11 +345,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       EpiTile et;
-      et.row0 = pt.m_blk * 2 * kBM + static_cast<int>(rank) * kBM;
-      et.row_end = p.rows;
+      et.row0 = pt.a_row0 + static_cast<int>(rank) * kBM;
+      et.row_end = pt.row_end;
       et.n0 = pt.n0;
-      et.sw0 = et.n0;
-      et.tma = true;   // dense: the bulk store clips at the tensor edge
+      et.sw0 = pt.sw0;
+      // The bulk store clips only at the tensor edge: used unless this CTA's
+      // slab crosses into the next expert's rows.
+      et.tma = !kGrouped || et.row0 + kBM <= et.row_end;
       epilogue_slab(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, pt.bn);
       tc_fence_before();
       __syncwarp();

@@ -139,11 +139,12 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x,
 fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* stream);
 
 /*
- * Tuning override for the dense linear (for measurement and tests; the
+ * Tuning override for the linear kernels (for measurement and tests; the
  * defaults are chosen per shape).  kernel_family: 0 = automatic, 1 = the
  * single-CTA kernel (128-row tiles), 2 = the CTA-pair kernel (256-row tiles,
- * tcgen05 cta_group::2), 3 = the swap-AB split-K cluster kernel (M <= 128
- * only; larger M falls back to automatic).  tile_n: 0 = automatic, else 128,
+ * tcgen05 cta_group::2; also selects it for the MoE grouped linear, whose
+ * default is single-CTA), 3 = the swap-AB
+ * split-K cluster kernel (M <= 128 only; larger M falls back to automatic).  tile_n: 0 = automatic, else 128,
  * 192, 256 or 512 (pair kernel only).  ksplit: 0 = automatic, else the split-K
  * cluster size 1, 2, 4 or 8 (split-K kernel only).  Process-wide; not thread-safe against
  * concurrent launches.  Environment variables FP8Q_FORCE_KERNEL

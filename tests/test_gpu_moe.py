@@ -47,7 +47,15 @@ def oracle_rows(Xg, offsets, W, rows):
     return out
 
 
-def test_small_groups_full_compare(fq):
+@pytest.fixture(params=[0, 2], ids=["single", "pair"])
+def family(request, fq):
+    """Grouped kernel family: 0 = automatic (single CTA, 128-row blocks), 2 = CTA pairs (256-row blocks)."""
+    fq.set_gemm_tuning(request.param, 0, 0)
+    yield request.param
+    fq.set_gemm_tuning(0, 0, 0)
+
+
+def test_small_groups_full_compare(fq, family):
     E, N, K = 6, 264, 272
     counts = [0, 130, 1, 0, 300, 57]
     off = wl.offsets_from_counts(counts)
@@ -67,8 +75,9 @@ def test_small_groups_full_compare(fq):
     [1, 1, 1, 1, 1, 1, 1, 1],     # single-row groups
     [128, 128, 256],              # exact tile multiples
     [700],                        # E = 1 behaves like a dense linear
+    [255, 257, 0, 1, 512, 100],   # 256-row blocks split one row before / after the boundary
 ])
-def test_adversarial_offsets(fq, counts):
+def test_adversarial_offsets(fq, family, counts):
     E, N, K = len(counts), 256, 256
     off = wl.offsets_from_counts(counts)
     R = int(off[-1])
@@ -79,7 +88,7 @@ def test_adversarial_offsets(fq, counts):
     assert_no_device_error()
 
 
-def test_bad_offsets_are_reported_and_nothing_written(fq):
+def test_bad_offsets_are_reported_and_nothing_written(fq, family):
     E, N, K = 3, 64, 128
     X = wl.random_f16((10, K), seed=1).cuda()
     Xq, s_x = fq.quantize_rows_dynamic(X)
@@ -99,7 +108,7 @@ def moe_case():
     return wl.moe()
 
 
-def test_moe_up_full(fq, moe_case):
+def test_moe_up_full(fq, family, moe_case):
     m = moe_case
     Y = run_gpu(fq, m.X_perm, m.offsets, m.W_up)
     rows = sample_rows(m.X_perm.shape[0], 256, seed=4)
@@ -107,7 +116,7 @@ def test_moe_up_full(fq, moe_case):
     assert_no_device_error()
 
 
-def test_moe_down_full(fq, moe_case):
+def test_moe_down_full(fq, family, moe_case):
     # Down projection on an independent seeded input of the up-output's shape.
     m = moe_case
     Xd = wl.random_f16((m.X_perm.shape[0], wl.MOE_F), seed=303)

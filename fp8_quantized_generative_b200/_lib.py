@@ -24,6 +24,7 @@ DEVERR_TIMEOUT_MMA = 0x2
 DEVERR_TIMEOUT_EPILOGUE = 0x4
 DEVERR_BAD_OFFSETS = 0x8
 DEVERR_TIMEOUT_CLUSTER = 0x10
+DEVERR_TIMEOUT_SELFTEST = 0x20
 
 
 class Fp8qError(RuntimeError):
@@ -48,6 +49,7 @@ SIGNATURES = {
     "fp8q_moe_grouped_linear": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_e4m3_encode_f32": (_INT, [_P, _I64, _P, _P]),
     "fp8q_set_gemm_tuning": (_INT, [_INT, _INT, _INT]),
+    "fp8q_selftest_wait_timeout": (_INT, [ctypes.c_uint32, _P]),
     "fp8q_device_error": (_INT, [_P, ctypes.POINTER(ctypes.c_uint32)]),
 }
 
@@ -110,6 +112,10 @@ def fp8q_e4m3_encode_f32(x, n, out, stream):
 
 def fp8q_set_gemm_tuning(kernel_family, tile_n, ksplit=0):
     return lib().fp8q_set_gemm_tuning(kernel_family, tile_n, ksplit)
+
+
+def fp8q_selftest_wait_timeout(limit_us, stream):
+    return lib().fp8q_selftest_wait_timeout(limit_us, stream)
 
 
 def fp8q_device_error(stream):

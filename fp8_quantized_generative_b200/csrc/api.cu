@@ -19,6 +19,20 @@
 #include "quant_rows.cuh"
 
 namespace fp8q {
+
+// Self-test of the bounded-wait machinery: one warp waits on an mbarrier that
+// nothing will ever arrive on, with the same wait routine the GEMMs use, and
+// must give up after `limit_ns` and report through the device error word.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0 && !mbar_wait_limit(&bar, 0, nullptr, limit_ns)) raise_error(0x20u);
+}
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -90,9 +104,18 @@ fp8q_status make_operand_map(CUtensorMap* m, const void* base, int64_t rows, int
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
+  // L2 promotion of operand loads; FP8Q_L2PROMO = 0 / 64 / 128 / 256 (default 256) for sweeps.
+  static const CUtensorMapL2promotion promo = [] {
+    const char* e = std::getenv("FP8Q_L2PROMO");
+    const int v = e ? std::atoi(e) : 256;
+    return v == 0 ? CU_TENSOR_MAP_L2_PROMOTION_NONE
+         : v == 64 ? CU_TENSOR_MAP_L2_PROMOTION_L2_64B
+         : v == 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                    : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+  }();
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     char buf[96];
     std::snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
@@ -452,6 +475,13 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
   // reused by every n-block while it is in L2, and the smaller B stays there.
   GemmParams q = p;
   q.n_fastest = int64_t(p.rows) > int64_t(p.N) ? 1 : 0;
+  // FP8Q_RASTER = 1 (m-blocks first) / 2 (n-blocks first) overrides the order for sweeps.
+  static const int raster = [] {
+    const char* e = std::getenv("FP8Q_RASTER");
+    return e ? std::atoi(e) : 0;
+  }();
+  if (raster == 1) q.n_fastest = 0;
+  if (raster == 2) q.n_fastest = 1;
   if (kn.force == 1) pair = false;
   if (kn.force == 2) pair = true;
   if (pair) {
@@ -610,6 +640,14 @@ fp8q_status fp8q_set_gemm_tuning(int kernel_family, int tile_n, int ksplit) {
   return FP8Q_OK;
 }
 
+fp8q_status fp8q_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 2000000u) return invalid("limit_us must be in [1, 2000000]");
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(uint64_t(limit_us) * 1000u);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "wait_timeout_selftest launch");
+  return FP8Q_OK;
+}
+
 fp8q_status fp8q_device_error(void* stream, uint32_t* flags) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
@@ -621,7 +659,7 @@ fp8q_status fp8q_device_error(void* stream, uint32_t* flags) {
   if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
   if (flags) *flags = v;
   if (v & (FP8Q_DEVERR_TIMEOUT_PRODUCER | FP8Q_DEVERR_TIMEOUT_MMA | FP8Q_DEVERR_TIMEOUT_EPILOGUE |
-           FP8Q_DEVERR_TIMEOUT_CLUSTER))
+           FP8Q_DEVERR_TIMEOUT_CLUSTER | FP8Q_DEVERR_TIMEOUT_SELFTEST))
     return FP8Q_ERR_TIMEOUT;
   if (v) return FP8Q_ERR_DEVICE_CHECK;
   return FP8Q_OK;

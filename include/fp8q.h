@@ -69,6 +69,7 @@ typedef enum {
 #define FP8Q_DEVERR_TIMEOUT_EPILOGUE 0x4u
 #define FP8Q_DEVERR_BAD_OFFSETS      0x8u
 #define FP8Q_DEVERR_TIMEOUT_CLUSTER  0x10u
+#define FP8Q_DEVERR_TIMEOUT_SELFTEST 0x20u
 
 /* Human-readable name of a status code.  Never returns NULL. */
 const char* fp8q_status_string(int status);
@@ -152,6 +153,16 @@ fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* 
  * 1, 2, 4 or 8) set the initial values.
  */
 fp8q_status fp8q_set_gemm_tuning(int kernel_family, int tile_n, int ksplit);
+
+/*
+ * Diagnostic: exercises the bounded-wait path every kernel relies on.  One
+ * warp waits on an mbarrier that nothing arrives on, with the same wait
+ * routine as the GEMM pipelines but a limit of `limit_us` microseconds
+ * (1 .. 2000000), gives up, sets FP8Q_DEVERR_TIMEOUT_SELFTEST and returns.
+ * The CUDA context stays usable; fp8q_device_error() then reports
+ * FP8Q_ERR_TIMEOUT.
+ */
+fp8q_status fp8q_selftest_wait_timeout(uint32_t limit_us, void* stream);
 
 /*
  * Synchronizes `stream`, then reads and clears the device error word of the

@@ -100,3 +100,8 @@ def test_python_wrappers_refuse_cpu_tensors():
     import fp8_quantized_generative_b200 as fq
     with pytest.raises(ValueError):
         fq.quantize_rows_dynamic(torch.zeros(4, 32, dtype=torch.float16))
+
+
+def test_selftest_rejects_bad_limits(L):
+    assert _lib.fp8q_selftest_wait_timeout(0, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_selftest_wait_timeout(3_000_000, 0) == _lib.FP8Q_ERR_INVALID_ARG

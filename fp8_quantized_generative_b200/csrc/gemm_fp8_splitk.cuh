@@ -12,11 +12,14 @@
 //     operand, so a single token still uses a full-height MMA;
 //   * the S CTAs of a cluster (cluster dims (S,1,1)) each take 1/S of the K
 //     blocks and accumulate a 128 x MPAD fp32 partial in TMEM;
-//   * S is 1, 2, 4 or 8; every CTA pushes the rows of its partial that CTA
-//     r owns (rows [r*128/S, (r+1)*128/S)) into CTA r's receive buffer with
-//     st.shared::cluster; after one cluster barrier CTA r sums its S slices
-//     locally in fixed rank order 0..S-1 (reproducible), applies the scales
-//     and writes fp16 -- no global scratch memory, no remote loads;
+//   * S is 1, 2, 4 or 8; CTA r owns weight rows [r*128/S, (r+1)*128/S) of
+//     the tile.  Each CTA stages its partial in its (now idle) load ring,
+//     slice by owner, and ships every other owner's slice with one bulk
+//     shared-memory-to-shared-memory copy (cp.async.bulk.shared::cluster)
+//     that completes on the owner's mbarrier; the owner then sums the S
+//     slices locally in fixed rank order 0..S-1 (reproducible), applies the
+//     scales (staged in shared memory beforehand) and writes fp16 -- no
+//     global scratch memory;
 //   * the weight tiles do not depend on the kernel launched before this one,
 //     so the first STAGES of them are requested before the programmatic-
 //     dependent-launch wait: their DRAM latency overlaps that kernel's tail.
@@ -34,14 +37,16 @@ struct SplitKLayout {
   static constexpr int kXBytes = MPAD * kBK;           // MPAD token rows
   static constexpr int kStageBytes = kWBytes + kXBytes;
   static constexpr int kRingBytes = STAGES * kStageBytes;
-  // Receive buffer: [S][128/S rows][MPAD + 4] fp32 = 128 rows of MPAD + 4
-  // words (16-byte aligned rows; the +4 keeps 8 consecutive rows of a
-  // 16-byte access on distinct bank groups).
+  // Partial rows of MPAD + 4 fp32 words (16-byte aligned rows; the +4 keeps
+  // 8 consecutive rows of a 16-byte access on distinct bank groups).
   static constexpr int kPitch = MPAD + 4;
-  static constexpr int kRecvBytes = kBM * kPitch * 4;
-  static constexpr int kNumBars = 2 * STAGES + 2;      // full, empty, tfull, drain
+  static constexpr int kPartBytes = kBM * kPitch * 4;  // send buffer (in the ring) and receive buffer
+  static_assert(kRingBytes >= kPartBytes, "the send buffer reuses the load ring");
+  static constexpr int kScaleFloats = 128 + MPAD;      // owner's s_w slice + the token scales
+  static constexpr int kNumBars = 2 * STAGES + 3;      // full, empty, tfull, drain, recv
   static constexpr int kTmemCols = MPAD < 32 ? 32 : MPAD;
-  static constexpr size_t kSmemBytes = 1024 + size_t(kRingBytes) + kRecvBytes + kNumBars * 8 + 32;
+  static constexpr size_t kSmemBytes =
+      1024 + size_t(kRingBytes) + kPartBytes + kScaleFloats * 4 + kNumBars * 8 + 32;
 };
 
 template <int MPAD, int STAGES>
@@ -57,12 +62,16 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sW = smem;
   uint8_t* sX = smem + STAGES * L::kWBytes;
+  float* send = reinterpret_cast<float*>(smem);                       // after the mainloop
   float* recv = reinterpret_cast<float*>(smem + L::kRingBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kRingBytes + L::kRecvBytes);
+  float* sc_w = reinterpret_cast<float*>(smem + L::kRingBytes + L::kPartBytes);   // 128
+  float* sc_x = sc_w + 128;                                                        // MPAD
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sc_x + MPAD);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* drain = bars + 2 * STAGES + 1;
+  uint64_t* recv_bar = bars + 2 * STAGES + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -76,6 +85,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   const int kb0 = static_cast<int>((int64_t(rank) * num_kb) / S);
   const int kb1 = static_cast<int>((int64_t(rank + 1) * num_kb) / S);
   const int nkb = kb1 - kb0;
+  const int SL = kBM / S;                          // weight rows owned by each CTA
+  const int mcols = (p.rows + 3) & ~3;             // token rows carried, rounded to 4
+  const uint32_t slice_bytes = static_cast<uint32_t>(SL * L::kPitch * 4);
 
   // Thread 0 is also the producer: it initializes the barriers and at once
   // requests the weight tiles of the first ring pass.  The weights do not
@@ -89,8 +101,11 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     }
     mbar_init(tfull, 1);
     mbar_init(drain, 1);
+    mbar_init(recv_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
+    // The S-1 peers' slices arrive as bulk copies counted on recv_bar.
+    mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(S - 1) * slice_bytes);
     for (int i = 0; i < pre; ++i) {
       mbar_arrive_expect_tx(&full[i], L::kStageBytes);
       tma_load_2d(sW + i * L::kWBytes, &tmW, &full[i], (kb0 + i) * kBK, n0);
@@ -176,12 +191,16 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     cluster_wait();
   } else {
     pdl_wait_prior_grid();
+    // Scales the reduction will need, staged while the mainloop runs.
+    const int et = threadIdx.x - kEpiWarp0 * 32;   // 0..127
+    {
+      const int n = n0 + rank * SL + et;
+      if (et < SL) sc_w[et] = n < p.N ? __ldg(p.s_w + n) : 0.0f;
+      if (et < p.rows) sc_x[et] = __ldg(p.s_x + et);
+    }
     // Partial: TMEM lane = weight row n of the tile, column = token row m.
-    // Row n belongs to CTA n / SL of the cluster, which receives it at slot
-    // [this rank][n % SL] of its receive buffer.
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    const int SL = kBM / S;
     bool have = nkb > 0;
     if (have && !mbar_wait(tfull, 0, abort_flag)) {
       raise_error(0x4u);
@@ -189,10 +208,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       have = false;
     }
     tc_fence_after();
-    cluster_wait();
-    const int owner = row / SL;
-    const uint32_t dst = mapa_shared(smem_u32(recv + (rank * SL + row % SL) * L::kPitch), static_cast<uint32_t>(owner));
-    const int mcols = (p.rows + 3) & ~3;   // token rows actually needed, rounded to 4
+    // Stage into the idle ring as [owner][row within owner][pitch].
+    float* dst = send + row * L::kPitch;
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     if (MPAD == 16) {
       uint32_t v[16];
@@ -203,8 +220,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 #pragma unroll
       for (int i = 0; i < 16; i += 4)
         if (i < mcols)
-          st_dsmem_v4(dst + i * 4, have ? __uint_as_float(v[i]) : 0.f, have ? __uint_as_float(v[i + 1]) : 0.f,
-                      have ? __uint_as_float(v[i + 2]) : 0.f, have ? __uint_as_float(v[i + 3]) : 0.f);
+          *reinterpret_cast<float4*>(dst + i) =
+              make_float4(have ? __uint_as_float(v[i]) : 0.f, have ? __uint_as_float(v[i + 1]) : 0.f,
+                          have ? __uint_as_float(v[i + 2]) : 0.f, have ? __uint_as_float(v[i + 3]) : 0.f);
     } else {
 #pragma unroll 1
       for (int c = 0; c < MPAD / 32; ++c) {
@@ -217,50 +235,57 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
           if (c * 32 + i < mcols)
-            st_dsmem_v4(dst + (c * 32 + i) * 4, have ? __uint_as_float(v[i]) : 0.f,
-                        have ? __uint_as_float(v[i + 1]) : 0.f, have ? __uint_as_float(v[i + 2]) : 0.f,
-                        have ? __uint_as_float(v[i + 3]) : 0.f);
+            *reinterpret_cast<float4*>(dst + c * 32 + i) =
+                make_float4(have ? __uint_as_float(v[i]) : 0.f, have ? __uint_as_float(v[i + 1]) : 0.f,
+                            have ? __uint_as_float(v[i + 2]) : 0.f, have ? __uint_as_float(v[i + 3]) : 0.f);
       }
     }
     tc_fence_before();
-  }
-
-  // Every push into every CTA's receive buffer is visible after this barrier;
-  // afterwards no CTA touches another's shared memory, so each may exit alone.
-  __syncthreads();
-  cluster_arrive();
-  cluster_wait();
-
-  if (warp >= kEpiWarp0) {
-    // This CTA owns weight rows [rank*SL, rank*SL + SL) of the tile: sum the
-    // S slices in rank order, scale, cast and store.  Four token rows per item.
-    const int SL = kBM / S;
-    const int t = threadIdx.x - kEpiWarp0 * 32;
-    const int m4n = (p.rows + 3) >> 2;
-    const int items = SL * m4n;
-    for (int idx = t; idx < items; idx += 128) {
-      const int nl = idx % SL;
-      const int m = (idx / SL) * 4;
-      const int n = n0 + rank * SL + nl;
-      if (n >= p.N) continue;
-      float4 acc = *reinterpret_cast<const float4*>(recv + nl * L::kPitch + m);
-      for (int s2 = 1; s2 < S; ++s2) {
-        const float4 v = *reinterpret_cast<const float4*>(recv + (s2 * SL + nl) * L::kPitch + m);
-        acc.x = __fadd_rn(acc.x, v.x);
-        acc.y = __fadd_rn(acc.y, v.y);
-        acc.z = __fadd_rn(acc.z, v.z);
-        acc.w = __fadd_rn(acc.w, v.w);
-      }
-      const float sw = __ldg(p.s_w + n);
-      const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+    fence_proxy_async_smem();
+    named_barrier(1, 128);   // the four epilogue warps have written the whole send buffer
+    cluster_wait();          // every CTA of the cluster is running (arrived at set-up)
+    if (et < S && et != rank) {
+      // ship owner et's rows to its receive slot [rank]
+      const uint32_t peer_recv = mapa_shared(smem_u32(recv + rank * SL * L::kPitch), static_cast<uint32_t>(et));
+      const uint32_t peer_bar = mapa_shared(smem_u32(recv_bar), static_cast<uint32_t>(et));
+      bulk_copy_to_cluster(peer_recv, send + et * SL * L::kPitch, slice_bytes, peer_bar);
+    }
+    // Own rows: wait for the S-1 peers' slices, sum in rank order, scale, store.
+    if (!mbar_wait(recv_bar, 0, abort_flag)) {
+      raise_error(0x10u);
+      *abort_flag = 1;
+    } else {
+      const int m4n = (p.rows + 3) >> 2;
+      const int items = SL * m4n;
+      for (int idx = et; idx < items; idx += 128) {
+        const int nl = idx % SL;
+        const int m = (idx / SL) * 4;
+        const int n = n0 + rank * SL + nl;
+        if (n >= p.N) continue;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s2 = 0; s2 < S; ++s2) {
+          const float* src = s2 == rank ? send + (rank * SL + nl) * L::kPitch : recv + (s2 * SL + nl) * L::kPitch;
+          const float4 v = *reinterpret_cast<const float4*>(src + m);
+          acc.x = __fadd_rn(acc.x, v.x);
+          acc.y = __fadd_rn(acc.y, v.y);
+          acc.z = __fadd_rn(acc.z, v.z);
+          acc.w = __fadd_rn(acc.w, v.w);
+        }
+        const float sw = sc_w[nl];
+        const float a[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (m + j < p.rows)
-          p.Y[static_cast<int64_t>(m + j) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(a[j], __ldg(p.s_x + m + j)), sw));
+        for (int j = 0; j < 4; ++j)
+          if (m + j < p.rows)
+            p.Y[static_cast<int64_t>(m + j) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(a[j], sc_x[m + j]), sw));
+      }
     }
   }
 
+  // No CTA may leave while a peer's bulk copy still reads its send buffer:
+  // every CTA arrives only after all copies into it have landed.
   __syncthreads();
+  cluster_arrive();
+  cluster_wait();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);

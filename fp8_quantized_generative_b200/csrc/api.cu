@@ -246,6 +246,18 @@ fp8q_status launch_gemm(const uint8_t* A, int64_t a_rows, const uint8_t* B, int6
   return FP8Q_OK;
 }
 
+// Split-K producers prefetch the rest of their weight slice into L2 at the
+// start (FP8Q_L2PF = 0 disables it, for sweeps).  Measured: a few percent
+// faster for one token row; the same idea slowed the grouped MoE kernel, so
+// only the split-K kernel uses it.
+int l2_prefetch_enabled() {
+  static const int v = [] {
+    const char* e = std::getenv("FP8Q_L2PF");
+    return (e && e[0] == '0') ? 0 : 1;
+  }();
+  return v;
+}
+
 // Per-device cache of how many 2-CTA clusters of a pair kernel fit at once.
 template <int BN, int STAGES, bool kGrouped>
 int max_pair_clusters(int dev) {
@@ -559,7 +571,7 @@ fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, 
   if (M == 0) return FP8Q_OK;
   if (!aligned16(Xq) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y_f16))
     return invalid("null or non-16-byte-aligned pointer");
-  GemmParams p;
+  GemmParams p = {};   // every field set below; zero for the rest
   p.s_x = s_x;
   p.s_w = s_w;
   p.Y = static_cast<__half*>(Y_f16);
@@ -571,6 +583,7 @@ fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, 
   p.n_fastest = 0;
   p.main_tiles = 0;
   p.tail_q = 1;
+  p.l2_prefetch = l2_prefetch_enabled();
   return launch_dense(Xq, Wq, p, static_cast<cudaStream_t>(stream));
 }
 
@@ -585,7 +598,7 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const i
   if (rows == 0) return FP8Q_OK;
   if (!aligned16(Xq) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y_f16))
     return invalid("null or non-16-byte-aligned pointer");
-  GemmParams p;
+  GemmParams p = {};   // every field set below; zero for the rest
   p.s_x = s_x;
   p.s_w = s_w;
   p.Y = static_cast<__half*>(Y_f16);
@@ -597,6 +610,7 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const i
   p.n_fastest = 0;
   p.main_tiles = 0;
   p.tail_q = 1;
+  p.l2_prefetch = l2_prefetch_enabled();
   // Single-CTA 128-row tiles by default; kernel family 2 selects CTA-pair
   // tiles of 256 expert rows (each weight tile read by half as many row
   // blocks), which measured no faster for the up projection and slower for

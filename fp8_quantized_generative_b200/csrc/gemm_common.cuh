@@ -39,6 +39,7 @@ struct GemmParams {
   // (tail_q in {1, 2, 4}) so that the last round keeps every cluster busy.
   int main_tiles;
   int tail_q;
+  int l2_prefetch;          // split-K: 1 = prefetch the rest of the weight slice into L2 at start
 };
 
 // One output slab of a CTA: 128 rows starting at row0, BN columns at n0.

@@ -110,6 +110,10 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       mbar_arrive_expect_tx(&full[i], L::kStageBytes);
       tma_load_2d(sW + i * L::kWBytes, &tmW, &full[i], (kb0 + i) * kBK, n0);
     }
+    // The rest of this CTA's weight slice goes to L2 now, so the whole
+    // stream is in flight from the start.
+    if (p.l2_prefetch)
+      for (int kb = kb0 + pre; kb < kb1; ++kb) tma_prefetch_l2_2d(&tmW, kb * kBK, n0);
     prefetch_tmap(&tmX);
   }
   if (warp == 1) {

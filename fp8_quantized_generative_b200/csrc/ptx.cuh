@@ -361,3 +361,13 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 }  // namespace fp8q
+
+namespace fp8q {
+// Pull a tensor tile into L2 ahead of its shared-memory load (no completion
+// tracking; deepens the DRAM requests in flight beyond the smem ring).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+}  // namespace fp8q

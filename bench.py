@@ -139,12 +139,14 @@ class ClockSampler:
 class Plan:
     """Device buffers (rotated sets) and the raw C-ABI launch sequence of one step."""
 
-    def __init__(self, kind, tensors, device, min_rotation_bytes):
+    def __init__(self, kind, tensors, device, min_rotation_bytes, fused=True):
         import fp8_quantized_generative_b200 as fq
         from fp8_quantized_generative_b200 import _lib
         self.fq, self.L = fq, _lib
         self.kind = kind
         self.device = device
+        # Up to 16 token rows the library quantizes inside the GEMM (one launch).
+        self.fused = fused and kind == "dense" and tensors[0].shape[0] <= fq.FUSED_MAX_ROWS
         if kind == "dense":
             X, W = tensors
             self.M, self.K = X.shape
@@ -188,12 +190,17 @@ class Plan:
         self.launches_per_step = len(self.kernels)
 
     def _kernel_names(self):
+        if self.fused:
+            return ["fp8_quantized_linear_fused"]
         if self.kind == "dense":
             return ["quant_rows", "fp8_gemm"]
         return ["quant_rows", "fp8_grouped_gemm_up", "quant_rows_h", "fp8_grouped_gemm_down"]
 
     def kernel_bytes_flops(self):
         """Algorithmic bytes and FLOPs of each launch of one step."""
+        if self.fused:
+            M, N, K = self.M, self.N, self.K
+            return [(2 * M * K + N * K + 4 * N + 2 * M * N, 2.0 * M * N * K)]
         if self.kind == "dense":
             M, N, K = self.M, self.N, self.K
             return [(M * K * 3 + 4 * M, 0.0),
@@ -208,7 +215,9 @@ class Plan:
         """Launch kernel k of step i (raw C ABI, integer pointers)."""
         L, p = self.L, self.bufs[i % self.sets]["p"]
         st = torch.cuda.current_stream(self.device).cuda_stream   # the capture stream inside a graph
-        if self.kind == "dense":
+        if self.fused:
+            s = L.fp8q_quantized_linear(p["X"], p["Wq"], p["sw"], self.M, self.N, self.K, p["Y"], 0, 0, st)
+        elif self.kind == "dense":
             if k == 0:
                 s = L.fp8q_quantize_rows_dynamic(p["X"], self.M, self.K, p["Xq"], p["sx"], st)
             else:
@@ -477,7 +486,7 @@ def run_ours(args, world, rank, local):
     desc, kind, tensors = workload_spec(args.workload)
     import fp8_quantized_generative_b200 as fq
     fq.set_gemm_tuning({"auto": 0, "single": 1, "pair": 2, "splitk": 3}[args.gemm], args.bn, args.ksplit)
-    plan = Plan(kind, tensors, device, min_rotation_bytes=3 * L2_BYTES)
+    plan = Plan(kind, tensors, device, min_rotation_bytes=3 * L2_BYTES, fused=args.fused)
     peaks, peak_src = load_peaks()
 
     sampler = ClockSampler(local)
@@ -543,6 +552,7 @@ def run_ours(args, world, rank, local):
                        "l2": f"rotating {plan.sets} buffer sets of {plan.bytes_per_set / 1e6:.0f} MB "
                              f"(> 3x 126 MB L2), no flush",
                        "step": " -> ".join(plan.kernels),
+                       "fused": plan.fused,
                        "launch": "per-call from the host" if args.no_graph else
                                  "CUDA graph of the K timed steps (replayed once untimed to upload)",
                        "kernel_timing": "per-kernel: CUDA events around a graph of that kernel's K launches"
@@ -594,6 +604,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of a CUDA graph")
+    ap.add_argument("--fused", action="store_true",
+                    help="one fused quantize+linear launch per step where it applies (<= 16 rows); "
+                         "default: the two launches, measured faster on B200")
     ap.add_argument("--gemm", default="auto", choices=["auto", "single", "pair", "splitk"],
                     help="dense GEMM kernel family (tuning sweeps; default: chosen per shape)")
     ap.add_argument("--bn", type=int, default=0, help="pair-kernel tile width (0 = automatic)")

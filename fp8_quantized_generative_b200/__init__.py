@@ -85,10 +85,32 @@ def linear(Xq: torch.Tensor, s_x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Ten
     return Y
 
 
-def quantized_linear(X: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor) -> torch.Tensor:
-    """fp16 activations in, fp16 out: per-token quantization then the FP8 linear."""
-    Xq, s_x = quantize_rows_dynamic(X)
-    return linear(Xq, s_x, Wq, s_w)
+FUSED_MAX_ROWS = 16
+
+
+def quantized_linear(X: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
+                     out: torch.Tensor | None = None, fused: bool = False) -> torch.Tensor:
+    """fp16 activations in, fp16 out: per-token quantization + FP8 linear +
+    dequantization.  fused=True runs one kernel (up to 16 rows, no workspace);
+    otherwise the two steps through a workspace allocated here."""
+    _need(X, torch.float16, "X", 2)
+    _need(Wq, torch.uint8, "Wq", 2)
+    _need(s_w, torch.float32, "s_w", 1)
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or s_w.shape[0] != N:
+        raise ValueError("shape mismatch")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X.device)
+    if fused and M <= FUSED_MAX_ROWS:
+        st = _lib.fp8q_quantized_linear(X.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K, Y.data_ptr(), 0, 0,
+                                        _stream(X))
+        if st == _lib.FP8Q_OK:
+            return Y
+    Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    s_x = torch.empty((M,), dtype=torch.float32, device=X.device)
+    check(_lib.fp8q_quantized_linear(X.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K, Y.data_ptr(),
+                                     Xq.data_ptr(), s_x.data_ptr(), _stream(X)), "fp8q_quantized_linear")
+    return Y
 
 
 def moe_grouped_linear(Xq: torch.Tensor, s_x: torch.Tensor, offsets: torch.Tensor, Wq: torch.Tensor,

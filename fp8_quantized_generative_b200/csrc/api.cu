@@ -150,6 +150,8 @@ fp8q_status make_output_map(CUtensorMap* m, const void* base, int64_t rows, int6
 }
 
 // ------------------------------------------------------------------ GEMM launch
+constexpr int kFusedMaxRows = 16;     // fused quantize + GEMM: token rows
+constexpr int kFusedMaxKBlocks = 32;  // ... and K blocks (of 128) per CTA
 constexpr int kBN = 256;        // single-CTA dense tiles (128 x 256)
 constexpr int kStages = 4;
 constexpr int kBNGrouped = 256; // MoE tiles (128 x 256); 128-wide tiles measured slower on B200
@@ -395,22 +397,24 @@ int choose_pair_bn(int64_t M, int64_t N, int clusters) {
 }
 
 // How many clusters of S CTAs of a split-K kernel fit on the device at once.
-template <int MPAD, int STAGES>
+template <int MPAD, int STAGES, bool kFused>
 int max_splitk_clusters(int dev, int S) {
   static int cache[kMaxDevices][9] = {};
   static std::mutex mu;
   std::lock_guard<std::mutex> g(mu);
   if (cache[dev][S] != 0) return cache[dev][S];
   using L = SplitKLayout<MPAD, STAGES>;
-  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES>;
-  if (ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES>>(L::kSmemBytes, dev) != cudaSuccess) {
+  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>;
+  const size_t max_smem = kFused ? L::fused_smem_bytes(kFusedMaxKBlocks) : L::kSmemBytes;
+  if (ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>>(max_smem, dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return -1;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S);
   cfg.blockDim = dim3(kSkThreads);
-  cfg.dynamicSmemBytes = L::kSmemBytes;
+  // occupancy at the shared memory of a typical launch (8 K blocks per CTA when fused)
+  cfg.dynamicSmemBytes = kFused ? L::fused_smem_bytes(8) : L::kSmemBytes;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
   attr.val.clusterDim.x = S;
@@ -427,43 +431,52 @@ int max_splitk_clusters(int dev, int S) {
   return n;
 }
 
-// Split factor: as many CTAs per 128-channel weight tile as keeps every
-// cluster of the grid resident at once (one wave), at most 8 and at most the
-// number of K blocks.
 // Split factor S in {1, 2, 4, 8} (a divisor of the 128 weight rows of a
 // tile, so each CTA of the cluster owns an equal slice of the reduction):
 // the largest that keeps every cluster of the grid resident at once (one
 // wave; two CTAs share an SM when their shared memory allows) and gives
 // each CTA at least one K block.
-template <int MPAD, int STAGES>
-int choose_ksplit(int dev, int sms, int n_tiles, int num_kb) {
-  (void)sms;
+template <int MPAD, int STAGES, bool kFused>
+int choose_ksplit(int dev, int n_tiles, int num_kb) {
   int S = 8;
   while (S > 1 && S > num_kb) S >>= 1;
   while (S > 1) {
-    const int fit = max_splitk_clusters<MPAD, STAGES>(dev, S);
+    const int fit = max_splitk_clusters<MPAD, STAGES, kFused>(dev, S);
     if (fit >= n_tiles) break;
     S >>= 1;
   }
   return S;
 }
 
-template <int MPAD, int STAGES>
-fp8q_status launch_splitk(const uint8_t* Xq, const uint8_t* Wq, const GemmParams& p, int dev, int sms,
-                          cudaStream_t st) {
+// Dense linear with at most 128 token rows.  kFused: A is the fp16
+// activations (p.x_f16) and the kernel quantizes them itself (<= 16 rows);
+// otherwise A is Xq with scales s_x.
+template <int MPAD, int STAGES, bool kFused>
+fp8q_status launch_splitk(const uint8_t* Xq, const uint8_t* Wq, const GemmParams& p, int dev, cudaStream_t st) {
   using L = SplitKLayout<MPAD, STAGES>;
   CUtensorMap tw, tx;
   fp8q_status s = make_operand_map(&tw, Wq, p.N, p.K, kBM);
   if (s != FP8Q_OK) return s;
-  s = make_operand_map(&tx, Xq, p.rows, p.K, MPAD);
-  if (s != FP8Q_OK) return s;
-  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES>;
-  cudaError_t e = ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES>>(L::kSmemBytes, dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(splitk)");
+  if (kFused) {
+    tx = tw;   // unused by the fused kernel
+  } else {
+    s = make_operand_map(&tx, Xq, p.rows, p.K, MPAD);
+    if (s != FP8Q_OK) return s;
+  }
   const int n_tiles = (p.N + kBM - 1) / kBM;
   const int num_kb = (p.K + kBK - 1) / kBK;
-  const int S = knobs().ksplit ? knobs().ksplit : choose_ksplit<MPAD, STAGES>(dev, sms, n_tiles, num_kb);
-  e = launch_ex(kernel, dim3(n_tiles * S), dim3(kSkThreads), L::kSmemBytes, st, S, true, tw, tx, p);
+  const int S = knobs().ksplit ? knobs().ksplit : choose_ksplit<MPAD, STAGES, kFused>(dev, n_tiles, num_kb);
+  const int nkb_max = (num_kb + S - 1) / S;
+  if (kFused && nkb_max > kFusedMaxKBlocks) {
+    g_last_error = "fused path: too many K blocks per CTA";
+    return FP8Q_ERR_UNSUPPORTED;
+  }
+  const size_t smem = kFused ? L::fused_smem_bytes(nkb_max) : L::kSmemBytes;
+  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>;
+  cudaError_t e = ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>>(
+      kFused ? L::fused_smem_bytes(kFusedMaxKBlocks) : L::kSmemBytes, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(splitk)");
+  e = launch_ex(kernel, dim3(n_tiles * S), dim3(kSkThreads), smem, st, S, true, tw, tx, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_splitk_kernel launch");
   return FP8Q_OK;
 }
@@ -477,10 +490,10 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
     // Up to 64 rows the stage count keeps shared memory under half an SM
     // (two CTAs resident), so the CTAs of the next kernel on the stream can
     // start and prefetch their weights while this one drains.
-    if (p.rows <= 16) return launch_splitk<16, 5>(Xq, Wq, p, dev, sms, st);
-    if (p.rows <= 32) return launch_splitk<32, 4>(Xq, Wq, p, dev, sms, st);
-    if (p.rows <= 64) return launch_splitk<64, 3>(Xq, Wq, p, dev, sms, st);
-    if (p.rows <= 128) return launch_splitk<128, 4>(Xq, Wq, p, dev, sms, st);
+    if (p.rows <= 16) return launch_splitk<16, 5, false>(Xq, Wq, p, dev, st);
+    if (p.rows <= 32) return launch_splitk<32, 4, false>(Xq, Wq, p, dev, st);
+    if (p.rows <= 64) return launch_splitk<64, 3, false>(Xq, Wq, p, dev, st);
+    if (p.rows <= 128) return launch_splitk<128, 4, false>(Xq, Wq, p, dev, st);
   }
   bool pair = p.rows > kBM;
   // Walk n-blocks first when A is the larger operand: each A block is then
@@ -585,6 +598,45 @@ fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, 
   p.tail_q = 1;
   p.l2_prefetch = l2_prefetch_enabled();
   return launch_dense(Xq, Wq, p, static_cast<cudaStream_t>(stream));
+}
+
+fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const float* s_w, int64_t M, int64_t N,
+                                  int64_t K, void* Y_f16, uint8_t* Xq_ws, float* s_x_ws, void* stream) {
+  if (M < 0 || M > kMaxDim) return invalid("M out of range");
+  if (N <= 0 || N > kMaxDim || N % 8 != 0) return invalid("N must be positive and a multiple of 8");
+  if (K <= 0 || K > kMaxDim || K % 16 != 0) return invalid("K must be positive and a multiple of 16");
+  if (M == 0) return FP8Q_OK;
+  if (!aligned16(X_f16) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y_f16))
+    return invalid("null or non-16-byte-aligned pointer");
+  const bool have_ws = Xq_ws != nullptr || s_x_ws != nullptr;
+  if (have_ws && (!aligned16(Xq_ws) || !aligned16(s_x_ws))) return invalid("workspace pointers must both be 16-byte aligned");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // With a workspace: the two launches (on B200 the faster choice -- the
+  // quantizer's launch and the GEMM's weight prefetch overlap through
+  // programmatic dependent launch, while the fused kernel must read whole
+  // fp16 rows for their maxima before its first MMA).  Without one: the
+  // fused kernel, up to 16 rows.
+  if (!have_ws && M <= kFusedMaxRows) {
+    int dev = 0, sms = 0;
+    const cudaError_t e = current_device_info(&dev, &sms);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    GemmParams p = {};
+    p.s_w = s_w;
+    p.Y = static_cast<__half*>(Y_f16);
+    p.x_f16 = static_cast<const __half*>(X_f16);
+    p.rows = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.E = 1;
+    p.tail_q = 1;
+    p.l2_prefetch = l2_prefetch_enabled();
+    const fp8q_status s = launch_splitk<16, 5, true>(nullptr, Wq, p, dev, st);
+    if (s != FP8Q_ERR_UNSUPPORTED) return s;   // else: too long a K slice, use the two-step path
+  }
+  if (!have_ws) return invalid("Xq_ws and s_x_ws are required for this shape (two-step path)");
+  fp8q_status s = fp8q_quantize_rows_dynamic(X_f16, M, K, Xq_ws, s_x_ws, stream);
+  if (s != FP8Q_OK) return s;
+  return fp8q_linear(Xq_ws, s_x_ws, Wq, s_w, M, N, K, Y_f16, stream);
 }
 
 fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const int32_t* offsets, int32_t E,

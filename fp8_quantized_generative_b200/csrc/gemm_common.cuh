@@ -29,6 +29,7 @@ struct GemmParams {
   const float* s_w;         // [E*N]
   __half* Y;                // [rows, N]
   const int32_t* offsets;   // [E+1] device, grouped only
+  const __half* x_f16;      // [rows, K] fp16 activations, fused quantize + GEMM only
   int rows;                 // M (dense) or total grouped rows
   int N;
   int K;

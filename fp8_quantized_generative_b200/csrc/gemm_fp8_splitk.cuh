@@ -20,12 +20,19 @@
 //     slices locally in fixed rank order 0..S-1 (reproducible), applies the
 //     scales (staged in shared memory beforehand) and writes fp16 -- no
 //     global scratch memory;
+//   * fused variant (kFused, at most 16 token rows): the kernel takes the
+//     fp16 activations, and each CTA computes the per-row maxima and scales
+//     itself (the same fp32 steps as quant_rows.cuh) and writes the E4M3
+//     codes of its K slice straight into the 128-byte-swizzled K-major
+//     shared-memory layout the MMA reads -- quantize + GEMM + dequantize in
+//     one launch ("FP8量化在生成式推荐系统OneRec-V2中的优化实践" §2.3);
 //   * the weight tiles do not depend on the kernel launched before this one,
 //     so the first STAGES of them are requested before the programmatic-
 //     dependent-launch wait: their DRAM latency overlaps that kernel's tail.
 #pragma once
 
 #include "gemm_common.cuh"
+#include "quant_rows.cuh"
 
 namespace fp8q {
 
@@ -43,13 +50,19 @@ struct SplitKLayout {
   static constexpr int kPartBytes = kBM * kPitch * 4;  // send buffer (in the ring) and receive buffer
   static_assert(kRingBytes >= kPartBytes, "the send buffer reuses the load ring");
   static constexpr int kScaleFloats = 128 + MPAD;      // owner's s_w slice + the token scales
-  static constexpr int kNumBars = 2 * STAGES + 3;      // full, empty, tfull, drain, recv
+  static constexpr int kNumBars = 2 * STAGES + 4;      // full, empty, tfull, drain, recv, xready
   static constexpr int kTmemCols = MPAD < 32 ? 32 : MPAD;
-  static constexpr size_t kSmemBytes =
-      1024 + size_t(kRingBytes) + kPartBytes + kScaleFloats * 4 + kNumBars * 8 + 32;
+  static constexpr int kBaseBytes = kRingBytes + kPartBytes + kScaleFloats * 4 + kNumBars * 8 + 32;
+  static constexpr size_t kSmemBytes = 1024 + size_t(kBaseBytes);
+  // Fused variant: 1024-aligned region after the base holding the E4M3 codes
+  // of the CTA's K blocks (MPAD x 128 bytes each) and the row statistics.
+  static constexpr int kFusedOffset = (kBaseBytes + 1023) & ~1023;
+  static size_t fused_smem_bytes(int nkb) {
+    return 1024 + size_t(kFusedOffset) + size_t(nkb) * kXBytes + 2 * MPAD * 4;
+  }
 };
 
-template <int MPAD, int STAGES>
+template <int MPAD, int STAGES, bool kFused>
 __global__ void __launch_bounds__(kSkThreads, 1)
     fp8_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                            const GemmParams p) {
@@ -72,6 +85,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* drain = bars + 2 * STAGES + 1;
   uint64_t* recv_bar = bars + 2 * STAGES + 2;
+  uint64_t* xready = bars + 2 * STAGES + 3;   // fused: the CTA's activation codes are in place
+  uint8_t* fz_codes = smem + L::kFusedOffset;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -88,6 +103,10 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   const int SL = kBM / S;                          // weight rows owned by each CTA
   const int mcols = (p.rows + 3) & ~3;             // token rows carried, rounded to 4
   const uint32_t slice_bytes = static_cast<uint32_t>(SL * L::kPitch * 4);
+  float* fz_amax = reinterpret_cast<float*>(fz_codes + nkb * L::kXBytes);
+  float* fz_r = fz_amax + MPAD;
+  // Fused: only the weight tiles travel through the ring.
+  constexpr uint32_t kLoadBytes = kFused ? L::kWBytes : L::kStageBytes;
 
   // Thread 0 is also the producer: it initializes the barriers and at once
   // requests the weight tiles of the first ring pass.  The weights do not
@@ -102,12 +121,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     mbar_init(tfull, 1);
     mbar_init(drain, 1);
     mbar_init(recv_bar, 1);
+    mbar_init(xready, 1);
     *abort_flag = 0;
     fence_barrier_init();
     // The S-1 peers' slices arrive as bulk copies counted on recv_bar.
     mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(S - 1) * slice_bytes);
     for (int i = 0; i < pre; ++i) {
-      mbar_arrive_expect_tx(&full[i], L::kStageBytes);
+      mbar_arrive_expect_tx(&full[i], kLoadBytes);
       tma_load_2d(sW + i * L::kWBytes, &tmW, &full[i], (kb0 + i) * kBK, n0);
     }
     // The rest of this CTA's weight slice goes to L2 now, so the whole
@@ -135,8 +155,10 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     if (lane == 0) {
       // The first ring pass of weight tiles is already in flight; the token
       // rows come from the previous kernel.
-      pdl_wait_prior_grid();
-      for (int i = 0; i < pre; ++i) tma_load_2d(sX + i * L::kXBytes, &tmX, &full[i], (kb0 + i) * kBK, 0);
+      if (!kFused) {
+        pdl_wait_prior_grid();
+        for (int i = 0; i < pre; ++i) tma_load_2d(sX + i * L::kXBytes, &tmX, &full[i], (kb0 + i) * kBK, 0);
+      }
       int s = pre % STAGES;
       uint32_t ph = pre == STAGES ? 1u : 0u;
       uint32_t armed = pre == STAGES ? (1u << STAGES) - 1u : (1u << pre) - 1u, armed_ph = 0;
@@ -146,9 +168,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+        mbar_arrive_expect_tx(&full[s], kLoadBytes);
         tma_load_2d(sW + s * L::kWBytes, &tmW, &full[s], kb * kBK, n0);
-        tma_load_2d(sX + s * L::kXBytes, &tmX, &full[s], kb * kBK, 0);
+        if (!kFused) tma_load_2d(sX + s * L::kXBytes, &tmX, &full[s], kb * kBK, 0);
         armed |= 1u << s;
         armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
         if (++s == STAGES) {
@@ -167,7 +189,12 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
+      if (kFused && !mbar_wait(xready, 0, abort_flag)) {
+        raise_error(0x2u);
+        *abort_flag = 1;
+        ok = false;
+      }
+      for (int kb = 0; kb < nkb && ok; ++kb) {
         if (!mbar_wait(&full[s], ph, abort_flag)) {
           raise_error(0x2u);
           *abort_flag = 1;
@@ -176,7 +203,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         }
         tc_fence_after();
         const uint64_t a0 = sw128_kmajor_desc(smem_u32(sW + s * L::kWBytes));
-        const uint64_t b0 = sw128_kmajor_desc(smem_u32(sX + s * L::kXBytes));
+        const uint64_t b0 = sw128_kmajor_desc(smem_u32(kFused ? fz_codes + kb * L::kXBytes : sX + s * L::kXBytes));
 #pragma unroll
         for (int k = 0; k < kBK / kUmmaK; ++k)
           mma_f8f6f4(tmem_base, a0 + static_cast<uint64_t>(k * kUmmaK / 16), b0 + static_cast<uint64_t>(k * kUmmaK / 16),
@@ -200,7 +227,51 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     {
       const int n = n0 + rank * SL + et;
       if (et < SL) sc_w[et] = n < p.N ? __ldg(p.s_w + n) : 0.0f;
-      if (et < p.rows) sc_x[et] = __ldg(p.s_x + et);
+      if (!kFused && et < p.rows) sc_x[et] = __ldg(p.s_x + et);
+    }
+    if (kFused) {
+      // Per-token dynamic quantization of the rows this CTA multiplies:
+      // row maxima over the whole K (warp w: rows w, w+4, ...), then the
+      // scales, then the codes of this CTA's K blocks in the swizzled
+      // layout of a 128-byte TMA box (row m at m*128, 16-byte chunk c at
+      // (c ^ (m & 7)) * 16).  Rows >= M and columns >= K are zero.
+      const int ew = warp - kEpiWarp0;
+      const int nvec = p.K >> 3;
+      for (int m = ew; m < p.rows; m += 4) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.x_f16 + static_cast<int64_t>(m) * p.K);
+        float a = 0.0f;
+        for (int j = lane; j < nvec; j += 32) a = absmax8(__ldg(src + j), a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if (lane == 0) fz_amax[m] = a;
+      }
+      named_barrier(1, 128);
+      if (et < p.rows) {
+        const RowScale rs = row_scale_from_amax(fz_amax[et]);
+        fz_r[et] = rs.r;
+        sc_x[et] = rs.s;
+      }
+      named_barrier(1, 128);
+      const int items = nkb * MPAD * 8;   // (k block, row, 16-byte chunk)
+      for (int it = et; it < items; it += 128) {
+        const int c = it & 7;
+        const int m = (it >> 3) % MPAD;
+        const int j = (it >> 3) / MPAD;
+        const int k = (kb0 + j) * kBK + c * 16;
+        uint4 out = make_uint4(0, 0, 0, 0);
+        if (m < p.rows && k < p.K) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.x_f16 + static_cast<int64_t>(m) * p.K + k);
+          const float r = fz_r[m];
+          const uint2 e0 = encode8(__ldg(src), r);
+          const uint2 e1 = encode8(__ldg(src + 1), r);
+          out = make_uint4(e0.x, e0.y, e1.x, e1.y);
+        }
+        st_shared_v4(smem_u32(fz_codes + j * L::kXBytes + m * kBK) + static_cast<uint32_t>((c ^ (m & 7)) << 4), out.x,
+                     out.y, out.z, out.w);
+      }
+      fence_proxy_async_smem();
+      named_barrier(1, 128);
+      if (et == 0) mbar_arrive(xready);
     }
     // Partial: TMEM lane = weight row n of the tile, column = token row m.
     const int q = warp & 3;

@@ -112,6 +112,24 @@ fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x,
                         void* Y_f16, void* stream);
 
 /*
+ * Quantize + FP8 linear + dequantize from fp16 activations  [P2 §2.3: the
+ * QuantizeLinear + GEMM + Dequantize fusion; P1 关键证据 steps 2-4].
+ *   X_f16 [M,K] fp16, Wq [N,K] uint8 and s_w [N] fp32 (per-channel
+ *   quantized weights) in;  Y_f16 [M,N] fp16 out.  Same results as
+ *   fp8q_quantize_rows_dynamic followed by fp8q_linear.
+ * With a workspace (Xq_ws [M,K] uint8 and s_x_ws [M] fp32, both non-NULL)
+ * the call runs the two steps through it (the workspace then holds the codes
+ * and scales); on B200 this is the faster choice.  With Xq_ws = s_x_ws = NULL
+ * and up to 16 token rows (K up to 4096 x the split factor) it is one fused
+ * kernel: each CTA computes the per-row scales and the E4M3 codes of its K
+ * slice in shared memory, so no intermediate touches HBM.  NULL workspace
+ * with a larger shape returns FP8Q_ERR_INVALID_ARG.
+ */
+fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const float* s_w,
+                                  int64_t M, int64_t N, int64_t K, void* Y_f16,
+                                  uint8_t* Xq_ws, float* s_x_ws, void* stream);
+
+/*
  * MoE expert grouped FP8 linear  [P1 关键证据 item 2: Sparse MoE grouped
  * GEMM; P2 §3.2 MoE acceleration].
  *   Xq [rows,K] uint8 and s_x [rows] fp32: token rows already grouped by

@@ -105,3 +105,16 @@ def test_python_wrappers_refuse_cpu_tensors():
 def test_selftest_rejects_bad_limits(L):
     assert _lib.fp8q_selftest_wait_timeout(0, 0) == _lib.FP8Q_ERR_INVALID_ARG
     assert _lib.fp8q_selftest_wait_timeout(3_000_000, 0) == _lib.FP8Q_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("M,N,K,ws", [
+    (-1, 16, 32, (0, 0)), (4, 12, 32, (0, 0)), (4, 16, 24, (0, 0)),
+    (4, 16, 32, (0x1000, 0)), (4, 16, 32, (0x1008, 0x1000)),
+])
+def test_quantized_linear_rejects(L, M, N, K, ws):
+    a = 0x1000
+    assert _lib.fp8q_quantized_linear(a, a, a, M, N, K, a, ws[0], ws[1], 0) == _lib.FP8Q_ERR_INVALID_ARG
+
+
+def test_quantized_linear_zero_rows_noop(L):
+    assert _lib.fp8q_quantized_linear(0, 0, 0, 0, 16, 32, 0, 0, 0, 0) == _lib.FP8Q_OK

@@ -48,6 +48,7 @@ SIGNATURES = {
     "fp8q_linear": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "fp8q_moe_grouped_linear": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_quantized_linear": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P]),
+    "fp8q_quantized_linear_noalloc": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "fp8q_e4m3_encode_f32": (_INT, [_P, _I64, _P, _P]),
     "fp8q_set_gemm_tuning": (_INT, [_INT, _INT, _INT]),
     "fp8q_selftest_wait_timeout": (_INT, [ctypes.c_uint32, _P]),
@@ -105,6 +106,10 @@ def fp8q_linear(Xq, s_x, Wq, s_w, M, N, K, Y, stream):
 
 def fp8q_quantized_linear(X, Wq, s_w, M, N, K, Y, Xq_ws, s_x_ws, stream):
     return lib().fp8q_quantized_linear(X, Wq, s_w, M, N, K, Y, Xq_ws, s_x_ws, stream)
+
+
+def fp8q_quantized_linear_noalloc(X, Wq, s_w, M, N, K, Y, stream):
+    return lib().fp8q_quantized_linear_noalloc(X, Wq, s_w, M, N, K, Y, stream)
 
 
 def fp8q_moe_grouped_linear(Xq, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream):

@@ -543,6 +543,40 @@ fp8q_status quantize(const void* X, int64_t M, int64_t K, uint8_t* Q, float* S, 
 }
 
 }  // namespace
+// ------------------------------------------------------------------ allocation-free variant
+// Scratch for fp8q_quantized_linear_noalloc: the E4M3 codes and per-row
+// scales that the two-step path keeps between its quantizer and its GEMM.
+// It is part of the library image, so every GPU that loads the library holds
+// these 8 MiB + 64 KiB until the process exits.
+constexpr size_t kNoAllocCodeBytes = size_t(8) << 20;    // M * K codes
+constexpr size_t kNoAllocScaleCount = size_t(16) << 10;  // M scales
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocCodeBytes + kNoAllocScaleCount * 4];
+
+// Device address of the scratch array, resolved once per device with that
+// device current (host code cannot use the array's name as a device pointer).
+static fp8q_status noalloc_scratch(uint8_t** out) {
+  struct Slot {
+    std::once_flag once;
+    uint8_t* ptr = nullptr;
+    cudaError_t err = cudaSuccess;
+  };
+  static Slot slots[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice, "device index");
+  Slot& sl = slots[dev];
+  std::call_once(sl.once, [&]() {
+    void* p = nullptr;
+    sl.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    sl.ptr = static_cast<uint8_t*>(p);
+  });
+  if (sl.err != cudaSuccess || sl.ptr == nullptr)
+    return cuda_fail(sl.err != cudaSuccess ? sl.err : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
+  *out = sl.ptr;
+  return FP8Q_OK;
+}
+
 }  // namespace fp8q
 
 using namespace fp8q;
@@ -637,6 +671,25 @@ fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const fl
   fp8q_status s = fp8q_quantize_rows_dynamic(X_f16, M, K, Xq_ws, s_x_ws, stream);
   if (s != FP8Q_OK) return s;
   return fp8q_linear(Xq_ws, s_x_ws, Wq, s_w, M, N, K, Y_f16, stream);
+}
+
+fp8q_status fp8q_quantized_linear_noalloc(const void* X_f16, const uint8_t* Wq, const float* s_w, int64_t M,
+                                          int64_t N, int64_t K, void* Y_f16, void* stream) {
+  if (M < 0 || M > kMaxDim) return invalid("M out of range");
+  if (N <= 0 || N > kMaxDim || N % 8 != 0) return invalid("N must be positive and a multiple of 8");
+  if (K <= 0 || K > kMaxDim || K % 16 != 0) return invalid("K must be positive and a multiple of 16");
+  if (M == 0) return FP8Q_OK;
+  if (M * K > int64_t(kNoAllocCodeBytes) || M > int64_t(kNoAllocScaleCount))
+    return invalid("fp8q_quantized_linear_noalloc: M*K must be <= 8388608 and M <= 16384 (fixed scratch size)");
+  if (!aligned16(X_f16) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y_f16))
+    return invalid("null or non-16-byte-aligned pointer");
+  uint8_t* scratch = nullptr;
+  const fp8q_status st = noalloc_scratch(&scratch);
+  if (st != FP8Q_OK) return st;
+  // codes at the start, scales after them; every call overwrites both in full
+  uint8_t* Xq = scratch;
+  float* s_x = reinterpret_cast<float*>(scratch + kNoAllocCodeBytes);
+  return fp8q_quantized_linear(X_f16, Wq, s_w, M, N, K, Y_f16, Xq, s_x, stream);
 }
 
 fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const int32_t* offsets, int32_t E,

@@ -130,6 +130,30 @@ fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const fl
                                   uint8_t* Xq_ws, float* s_x_ws, void* stream);
 
 /*
+ * Allocation-free form of fp8q_quantized_linear (the pages have no
+ * counterpart; this is a deployment convenience).  Same inputs, output and
+ * numerics as fp8q_quantized_linear with a workspace, but the codes and
+ * scales between the quantizer and the GEMM live in a fixed scratch array
+ * built into the library, so the caller passes only X, the quantized weights
+ * and Y.  It is for callers that cannot call cudaMalloc -- for example code
+ * running inside a host framework that owns all device memory through its own
+ * pre-sized pool, or a serving loop that must never trigger an allocation
+ * (and the device synchronization it can cause) once it is running.
+ *   Limits: M*K <= 8388608 and M <= 16384, else FP8Q_ERR_INVALID_ARG with an
+ *   explanatory message (fp8q_last_error_message()).  The scratch costs every
+ *   GPU that loads the library 8 MiB + 64 KiB of device memory until exit.
+ *   The first call on a device looks up the scratch address for that device
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture on the device.
+ *   All calls on a device share the one scratch array and nothing in it needs
+ *   to start at zero (each call overwrites the codes and scales it reads);
+ *   two calls whose work overlaps on the GPU (different streams without
+ *   ordering) race on it and give wrong results.  No call allocates memory.
+ */
+fp8q_status fp8q_quantized_linear_noalloc(const void* X_f16, const uint8_t* Wq, const float* s_w,
+                                          int64_t M, int64_t N, int64_t K, void* Y_f16, void* stream);
+
+/*
  * MoE expert grouped FP8 linear  [P1 关键证据 item 2: Sparse MoE grouped
  * GEMM; P2 §3.2 MoE acceleration].
  *   Xq [rows,K] uint8 and s_x [rows] fp32: token rows already grouped by

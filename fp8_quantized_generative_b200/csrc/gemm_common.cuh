@@ -61,35 +61,83 @@ __device__ __forceinline__ uint32_t stage_off(int r, int c) {
   return static_cast<uint32_t>(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
 }
 
-// One epilogue warp drains its 32 TMEM lanes (rows q*32 .. q*32+31 of the
-// slab, q = warp % 4 as tcgen05.ld requires) over its half of the BN columns,
-// 32 columns at a time: TMEM -> registers -> scale and cast -> swizzled
-// staging tile in shared memory -> one bulk tensor store (or, for a slab cut
-// by an expert boundary, coalesced row-masked stores).
-// `bn` is the slab width (a multiple of 64; each warp takes bn/2 columns).
-__device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams& p, const CUtensorMap* tmY,
-                                              uint32_t tmem_acc, int warp, int lane, uint8_t* stage, int bn) {
+// The scales one epilogue lane applies to a slab: s_x of its row and, for
+// each 32-column chunk of its warp, s_w of column (chunk start + lane).
+template <int kMaxChunks>
+struct EpiScales {
+  float sx;
+  float sw[kMaxChunks];
+};
+
+template <int kMaxChunks>
+__device__ __forceinline__ EpiScales<kMaxChunks> epilogue_scales(const EpiTile& t, const GemmParams& p, int warp,
+                                                                 int lane, int bn) {
+  EpiScales<kMaxChunks> e;
   const int q = warp & 3;
   const int h = (warp - kEpiWarp0) >> 2;
   const int r = t.row0 + q * 32 + lane;
-  const float sx = r < t.row_end ? __ldg(p.s_x + r) : 0.0f;
+  e.sx = r < t.row_end ? __ldg(p.s_x + r) : 0.0f;
+#pragma unroll
+  for (int j = 0; j < kMaxChunks; ++j) {
+    const int cl = h * (bn / 2) + j * 32 + lane;
+    e.sw[j] = (j < bn / 64 && t.n0 + cl < p.N) ? __ldg(p.s_w + t.sw0 + cl) : 0.0f;
+  }
+  return e;
+}
+
+// One epilogue warp drains its 32 TMEM lanes (rows q*32 .. q*32+31 of the
+// slab, q = warp % 4 as tcgen05.ld requires) over its half of the bn columns,
+// 32 columns at a time: TMEM -> registers -> scale and cast -> swizzled
+// staging tile in shared memory -> one bulk tensor store (or, for a slab cut
+// by an expert boundary, coalesced row-masked stores).
+// `bn` is the slab width (a multiple of 64, at most 64 * kMaxChunks; each
+// warp takes bn/2 columns).
+//
+// Two paces.  While the MMAs of the next tile run (kDrain = false) each chunk
+// fetches its weight scales and waits for its TMEM load before the next one
+// starts; a faster epilogue there was measured to slow the concurrent MMAs
+// by about 3% (it competes with them for the SM's shared-memory and TMEM
+// traffic), more than it saves.  For a CTA's last tile (kDrain = true)
+// nothing else runs: the scales `pre` were loaded before the accumulator
+// wait, and the TMEM load of chunk j+1 is in flight while chunk j is scaled
+// and stored, which shortens the exposed final epilogue by about a third.
+template <int kMaxChunks, bool kDrain>
+__device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams& p, const CUtensorMap* tmY,
+                                              uint32_t tmem_acc, int warp, int lane, uint8_t* stage, int bn,
+                                              const EpiScales<kMaxChunks>& pre) {
+  const int q = warp & 3;
+  const int h = (warp - kEpiWarp0) >> 2;
+  const int nch = bn / 64;
+  const int r = t.row0 + q * 32 + lane;
+  const float sx = kDrain ? pre.sx : (r < t.row_end ? __ldg(p.s_x + r) : 0.0f);
   const uint32_t sbase = smem_u32(stage);
   const uint32_t taddr0 = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * (bn / 2));
-#pragma unroll 1
-  for (int j = 0; j < bn / 64; ++j) {
-    const int cl = h * (bn / 2) + j * 32;   // first column of the chunk within the tile
-    const int colw = t.n0 + cl + lane;
-    const float sw_lane = colw < p.N ? __ldg(p.s_w + t.sw0 + cl + lane) : 0.0f;
-    uint32_t v[32];
-    tmem_ld_32x32b_x32(taddr0 + static_cast<uint32_t>(j * 32), v);
-    tmem_ld_wait();
+  uint32_t v[2][32];
+  if (kDrain) {
+    tmem_ld_32x32b_x32(taddr0, v[0]);
+    tmem_ld_wait_regs(v[0]);
+  }
+#pragma unroll
+  for (int j = 0; j < kMaxChunks; ++j) {
+    if (j >= nch) break;
+    const int cl = h * (bn / 2) + j * 32;   // first column of the chunk within the slab
+    uint32_t* cur = v[kDrain ? (j & 1) : 0];
+    float sw_lane;
+    if (kDrain) {
+      sw_lane = pre.sw[j];
+      if (j + 1 < nch) tmem_ld_32x32b_x32(taddr0 + static_cast<uint32_t>((j + 1) * 32), v[(j + 1) & 1]);
+    } else {
+      sw_lane = t.n0 + cl + lane < p.N ? __ldg(p.s_w + t.sw0 + cl + lane) : 0.0f;
+      tmem_ld_32x32b_x32(taddr0 + static_cast<uint32_t>(j * 32), v[0]);
+      tmem_ld_wait_regs(v[0]);
+    }
     uint32_t packed[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float w0 = __shfl_sync(0xffffffffu, sw_lane, 2 * i);
       const float w1 = __shfl_sync(0xffffffffu, sw_lane, 2 * i + 1);
-      const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * i]), sx), w0);
-      const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * i + 1]), sx), w1);
+      const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i]), sx), w0);
+      const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i + 1]), sx), w1);
       const __half2 hv = __floats2half2_rn(y0, y1);
       packed[i] = *reinterpret_cast<const uint32_t*>(&hv);
     }
@@ -120,6 +168,7 @@ __device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams
       }
       __syncwarp();
     }
+    if (kDrain && j + 1 < nch) tmem_ld_wait_regs(v[(j + 1) & 1]);
   }
 }
 

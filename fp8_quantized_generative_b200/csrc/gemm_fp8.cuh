@@ -268,12 +268,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_ph = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const TileCoord c = decode_tile<kGrouped, BN>(t, p, num_m, num_n, tile_prefix, offs);
-      if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
-        raise_error(0x4u);
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
       EpiTile et;
       et.row0 = c.a_row0;
       et.row_end = c.row_end;
@@ -282,7 +276,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // A bulk store clips only at the tensor edge, so it is used unless the
       // slab crosses into the next expert's rows.
       et.tma = !kGrouped || c.a_row0 + kBM <= c.row_end;
-      epilogue_slab(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, BN);
+      // The CTA's last tile: its epilogue is exposed, so it runs at the drain pace.
+      const bool last_tile = t + static_cast<int>(gridDim.x) >= total;
+      EpiScales<BN / 64> sc{};
+      if (last_tile) sc = epilogue_scales<BN / 64>(et, p, warp, lane, BN);
+      if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
+        raise_error(0x4u);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      if (last_tile)
+        epilogue_slab<BN / 64, true>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, BN, sc);
+      else
+        epilogue_slab<BN / 64, false>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, BN, sc);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);

@@ -338,12 +338,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_ph = 0;
     for (int t = pair; t < total; t += npairs) {
       const PairTile pt = pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs);
-      if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
-        raise_error(0x4u);
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
       EpiTile et;
       et.row0 = pt.a_row0 + static_cast<int>(rank) * kBM;
       et.row_end = pt.row_end;
@@ -352,7 +346,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // The bulk store clips only at the tensor edge: used unless this CTA's
       // slab crosses into the next expert's rows.
       et.tma = !kGrouped || et.row0 + kBM <= et.row_end;
-      epilogue_slab(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, pt.bn);
+      // The CTA's last tile: its epilogue is exposed, so it runs at the drain pace.
+      const bool last_tile = t + static_cast<int>(npairs) >= total;
+      EpiScales<BN / 64> sc{};
+      if (last_tile) sc = epilogue_scales<BN / 64>(et, p, warp, lane, pt.bn);
+      if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
+        raise_error(0x4u);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      if (last_tile)
+        epilogue_slab<BN / 64, true>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, pt.bn, sc);
+      else
+        epilogue_slab<BN / 64, false>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, pt.bn, sc);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);

@@ -159,6 +159,20 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Wait for outstanding tcgen05.ld and make every later use of `v` depend on
+// the wait: the empty statement "rewrites" the registers after it, so no
+// computation on them can be scheduled above the wait even when another load
+// was issued in between (double-buffered TMEM reads).
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&v)[32]) {
+  tmem_ld_wait();
+  asm volatile(""
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                 "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                 "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
+                 "+r"(v[29]), "+r"(v[30]), "+r"(v[31]));
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile stored the way a
 // TMA 128-byte-swizzled load leaves it: rows of 128 bytes, 8-row (1024-byte)
 // swizzle atoms stacked along M/N.  Fields (tcgen05 matrix descriptor):

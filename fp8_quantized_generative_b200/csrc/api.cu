@@ -165,6 +165,7 @@ struct Knobs {
   int force = 0;  // 0 auto, 1 single, 2 pair, 3 split-K (M <= 128)
   int bn = 0;
   int ksplit = 0; // split-K cluster size, 0 = automatic
+  int half_tiles = 1; // FP8Q_HALF_TILES: 0 = CTA-pair grouped kernel uses only M = 256 tiles
 };
 Knobs& knobs() {
   static Knobs k = []() {
@@ -176,6 +177,7 @@ Knobs& knobs() {
     }
     if (const char* k = std::getenv("FP8Q_KSPLIT")) r.ksplit = std::atoi(k);
     if (const char* b = std::getenv("FP8Q_BN")) r.bn = std::atoi(b);
+    if (const char* h = std::getenv("FP8Q_HALF_TILES")) r.half_tiles = h[0] == '0' ? 0 : 1;
     return r;
   }();
   return k;
@@ -348,9 +350,16 @@ fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, int64_t b_rows, cons
     p.tail_q = ts.q;
     tiles = int64_t(ts.main_tiles) + (full - ts.main_tiles) * ts.q;
   }
-  CUtensorMap ta, tb, tbt, ty;
+  CUtensorMap ta, tah, tb, tbt, ty;
   fp8q_status s = make_operand_map(&ta, A, p.rows, p.K, kBM);
   if (s != FP8Q_OK) return s;
+  if (kGrouped) {
+    // half tiles: 64 rows of A per CTA
+    s = make_operand_map(&tah, A, p.rows, p.K, kBM / 2);
+    if (s != FP8Q_OK) return s;
+  } else {
+    tah = ta;   // unused
+  }
   s = make_operand_map(&tb, B, b_rows, p.K, L::kWide ? 128 : L::kBRows);
   if (s != FP8Q_OK) return s;
   s = make_operand_map(&tbt, B, b_rows, p.K, L::kWide ? 128 : L::kBRows / ts.q);
@@ -362,8 +371,8 @@ fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, int64_t b_rows, cons
       L::smem_bytes(kGrouped ? kMaxExperts : 0), dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair)");
   const int pairs = static_cast<int>(tiles < clusters ? (tiles < 1 ? 1 : tiles) : clusters);
-  e = launch_ex(kernel, dim3(2 * pairs), dim3(kGemmThreads), L::smem_bytes(kGrouped ? p.E : 0), st, 2, true, ta, tb,
-                tbt, ty, p);
+  e = launch_ex(kernel, dim3(2 * pairs), dim3(kGemmThreads), L::smem_bytes(kGrouped ? p.E : 0), st, 2, true, ta, tah,
+                tb, tbt, ty, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_pair_kernel launch");
   return FP8Q_OK;
 }
@@ -514,7 +523,7 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
     int bn = kn.bn ? kn.bn : choose_pair_bn(p.rows, p.N, clusters > 0 ? clusters : sms / 2);
     switch (bn) {
       case 128: return launch_pair<128, 8, false>(Xq, Wq, p.N, q, dev, st);
-      case 192: return launch_pair<192, 7, false>(Xq, Wq, p.N, q, dev, st);
+      case 192: return launch_pair<192, 6, false>(Xq, Wq, p.N, q, dev, st);
       case 512: return launch_pair<512, 4, false>(Xq, Wq, p.N, q, dev, st);
       default: return launch_pair<256, 6, false>(Xq, Wq, p.N, q, dev, st);
     }
@@ -716,6 +725,7 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const i
   p.main_tiles = 0;
   p.tail_q = 1;
   p.l2_prefetch = l2_prefetch_enabled();
+  p.half_tiles = knobs().half_tiles;
   // Single-CTA 128-row tiles by default; kernel family 2 selects CTA-pair
   // tiles of 256 expert rows (each weight tile read by half as many row
   // blocks), which measured no faster for the up projection and slower for
@@ -725,7 +735,7 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const i
     const cudaError_t e = current_device_info(&dev, &sms);
     if (e != cudaSuccess) return cuda_fail(e, "device query");
     const int64_t tiles = ((rows + 2 * kBM - 1) / (2 * kBM) + E) * ((N + 255) / 256);
-    return launch_pair<256, 6, true>(Xq, Wq, int64_t(E) * N, p, dev, static_cast<cudaStream_t>(stream), tiles);
+    return launch_pair<256, 5, true>(Xq, Wq, int64_t(E) * N, p, dev, static_cast<cudaStream_t>(stream), tiles);
   }
   const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBNGrouped - 1) / kBNGrouped);
   return launch_gemm<true>(Xq, rows, Wq, int64_t(E) * N, p, tiles, static_cast<cudaStream_t>(stream));

@@ -21,7 +21,9 @@ constexpr int kEpiWarp0 = 2;      // warps 0, 1: TMA producer, MMA issuer
 constexpr int kEpiWarps = 8;      // two epilogue warps per TMEM lane quadrant
 constexpr int kGemmThreads = (kEpiWarp0 + kEpiWarps) * 32;
 constexpr int kStageTileBytes = 32 * 32 * 2;   // one 32 x 32 fp16 output tile per epilogue warp
-constexpr int kEpiSmemBytes = kEpiWarps * kStageTileBytes;
+// Staging for kBufs tiles per epilogue warp: buffer b of warp w at
+// (b * kEpiWarps + w) * kStageTileBytes.
+__host__ __device__ constexpr int epi_smem_bytes(int bufs) { return bufs * kEpiWarps * kStageTileBytes; }
 constexpr int kMaxExperts = 1024;
 
 struct GemmParams {
@@ -41,6 +43,7 @@ struct GemmParams {
   int main_tiles;
   int tail_q;
   int l2_prefetch;          // split-K: 1 = prefetch the rest of the weight slice into L2 at start
+  int half_tiles;           // CTA-pair grouped kernel: an expert's last <= 128 rows as an M = 128 pair tile
 };
 
 // One output slab of a CTA: 128 rows starting at row0, BN columns at n0.
@@ -49,7 +52,7 @@ struct EpiTile {
   int row_end;   // rows >= row_end are not stored
   int n0;
   int sw0;       // index into s_w of column n0
-  bool tma;      // the bulk tensor store may write the whole slab
+  bool clip;     // rows >= row_end lie past the output tensor, where a bulk store clips them
 };
 
 // Staging layout of a 32 x 32 fp16 tile: row r occupies 64 bytes, its four
@@ -61,8 +64,42 @@ __device__ __forceinline__ uint32_t stage_off(int r, int c) {
   return static_cast<uint32_t>(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
 }
 
-// The scales one epilogue lane applies to a slab: s_x of its row and, for
-// each 32-column chunk of its warp, s_w of column (chunk start + lane).
+// What one epilogue warp drains: 32 output rows from qrow0, nch chunks of
+// 32 columns from column col0 of the tile, held in the warp's TMEM lane
+// quadrant (q = warp % 4, as tcgen05.ld requires) from TMEM column tcol0.
+// Normal tiles: quadrant q holds rows q*32.. of the CTA's 128-row slab and
+// the two warps of a quadrant split the bn columns.  Half tiles (a CTA-pair
+// MMA with M = 128: 64 rows per CTA) keep the slab's 64 rows twice: lanes
+// 0-63 hold columns 0..bn/2-1 and lanes 64-127 columns bn/2..bn-1, both at
+// TMEM columns 0..bn/2-1 (measured on B200 with a layout probe).
+struct EpiWarpView {
+  int qrow0;
+  int col0;
+  int tcol0;
+  int nch;
+};
+
+__device__ __forceinline__ EpiWarpView epi_view(const EpiTile& t, int warp, int bn, bool half) {
+  const int q = warp & 3;
+  const int h = (warp - kEpiWarp0) >> 2;
+  EpiWarpView v;
+  if (!half) {
+    v.qrow0 = t.row0 + q * 32;
+    v.col0 = h * (bn / 2);
+    v.tcol0 = h * (bn / 2);
+    v.nch = bn / 64;
+  } else {
+    v.qrow0 = t.row0 + (q & 1) * 32;
+    v.col0 = (q >> 1) * (bn / 2) + h * (bn / 4);
+    v.tcol0 = h * (bn / 4);
+    v.nch = bn / 128;
+  }
+  return v;
+}
+
+// The scales one epilogue lane applies: s_x of its row and, for each 32-column
+// chunk of its warp, s_w of column (chunk start + lane).  Loaded before the
+// wait for the accumulator, so their latency hides behind the tile's MMAs.
 template <int kMaxChunks>
 struct EpiScales {
   float sx;
@@ -70,88 +107,83 @@ struct EpiScales {
 };
 
 template <int kMaxChunks>
-__device__ __forceinline__ EpiScales<kMaxChunks> epilogue_scales(const EpiTile& t, const GemmParams& p, int warp,
-                                                                 int lane, int bn) {
+__device__ __forceinline__ EpiScales<kMaxChunks> epilogue_scales(const EpiTile& t, const GemmParams& p,
+                                                                 const EpiWarpView& w, int lane) {
   EpiScales<kMaxChunks> e;
-  const int q = warp & 3;
-  const int h = (warp - kEpiWarp0) >> 2;
-  const int r = t.row0 + q * 32 + lane;
+  const int r = w.qrow0 + lane;
   e.sx = r < t.row_end ? __ldg(p.s_x + r) : 0.0f;
 #pragma unroll
   for (int j = 0; j < kMaxChunks; ++j) {
-    const int cl = h * (bn / 2) + j * 32 + lane;
-    e.sw[j] = (j < bn / 64 && t.n0 + cl < p.N) ? __ldg(p.s_w + t.sw0 + cl) : 0.0f;
+    const int cl = w.col0 + j * 32 + lane;
+    e.sw[j] = (j < w.nch && t.n0 + cl < p.N) ? __ldg(p.s_w + t.sw0 + cl) : 0.0f;
   }
   return e;
 }
 
-// One epilogue warp drains its 32 TMEM lanes (rows q*32 .. q*32+31 of the
-// slab, q = warp % 4 as tcgen05.ld requires) over its half of the bn columns,
-// 32 columns at a time: TMEM -> registers -> scale and cast -> swizzled
-// staging tile in shared memory -> one bulk tensor store (or, for a slab cut
-// by an expert boundary, coalesced row-masked stores).
-// `bn` is the slab width (a multiple of 64, at most 64 * kMaxChunks; each
-// warp takes bn/2 columns).
-//
-// Two paces.  While the MMAs of the next tile run (kDrain = false) each chunk
-// fetches its weight scales and waits for its TMEM load before the next one
-// starts; a faster epilogue there was measured to slow the concurrent MMAs
-// by about 3% (it competes with them for the SM's shared-memory and TMEM
-// traffic), more than it saves.  For a CTA's last tile (kDrain = true)
-// nothing else runs: the scales `pre` were loaded before the accumulator
-// wait, and the TMEM load of chunk j+1 is in flight while chunk j is scaled
-// and stored, which shortens the exposed final epilogue by about a third.
-template <int kMaxChunks, bool kDrain>
+// One epilogue warp drains its view (above), 32 columns at a time:
+// TMEM -> registers -> scale and cast -> swizzled staging tile in shared
+// memory -> one bulk tensor store.  A warp whose 32 rows all lie past row_end
+// does nothing; one whose rows straddle row_end inside the tensor (an MoE
+// expert boundary) stores its valid rows with coalesced masked stores
+// instead of the bulk store.
+// The scales `pre` were loaded before the accumulator wait, the TMEM load of
+// chunk j+1 is in flight while chunk j is scaled and stored, and with two
+// staging tiles per warp (kBufs = 2) chunk j+1 is written while the bulk
+// store of chunk j still reads its tile.  (A slower variant that fetched the
+// scales per chunk and waited out every load and store measured no faster
+// on the dense shapes and up to 12% slower on the MoE kernels.)
+// w.nch <= kMaxChunks.
+template <int kMaxChunks, int kBufs>
 __device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams& p, const CUtensorMap* tmY,
-                                              uint32_t tmem_acc, int warp, int lane, uint8_t* stage, int bn,
-                                              const EpiScales<kMaxChunks>& pre) {
+                                              uint32_t tmem_acc, const EpiWarpView& w, int warp, int lane,
+                                              uint8_t* stage, const EpiScales<kMaxChunks>& pre) {
+  static_assert(kBufs == 1 || kBufs == 2, "staging buffers");
   const int q = warp & 3;
-  const int h = (warp - kEpiWarp0) >> 2;
-  const int nch = bn / 64;
-  const int r = t.row0 + q * 32 + lane;
-  const float sx = kDrain ? pre.sx : (r < t.row_end ? __ldg(p.s_x + r) : 0.0f);
-  const uint32_t sbase = smem_u32(stage);
-  const uint32_t taddr0 = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * (bn / 2));
+  const int nch = w.nch;
+  const int qrow0 = w.qrow0;
+  const int valid = t.row_end - qrow0;   // rows of this warp that are stored (<= 0: none)
+  if (valid <= 0) return;
+  const bool bulk = t.clip || valid >= 32;
+  const uint32_t taddr0 = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(w.tcol0);
   uint32_t v[2][32];
-  if (kDrain) {
-    tmem_ld_32x32b_x32(taddr0, v[0]);
-    tmem_ld_wait_regs(v[0]);
-  }
+  tmem_ld_32x32b_x32(taddr0, v[0]);
+  // Buffer j & 1 below assumes no store of an earlier slab still reads
+  // either tile (that slab's last store was issued a whole mainloop ago).
+  if (kBufs == 2 && lane == 0) bulk_wait_read_all();
+  tmem_ld_wait_regs(v[0]);
 #pragma unroll
   for (int j = 0; j < kMaxChunks; ++j) {
     if (j >= nch) break;
-    const int cl = h * (bn / 2) + j * 32;   // first column of the chunk within the slab
-    uint32_t* cur = v[kDrain ? (j & 1) : 0];
-    float sw_lane;
-    if (kDrain) {
-      sw_lane = pre.sw[j];
-      if (j + 1 < nch) tmem_ld_32x32b_x32(taddr0 + static_cast<uint32_t>((j + 1) * 32), v[(j + 1) & 1]);
-    } else {
-      sw_lane = t.n0 + cl + lane < p.N ? __ldg(p.s_w + t.sw0 + cl + lane) : 0.0f;
-      tmem_ld_32x32b_x32(taddr0 + static_cast<uint32_t>(j * 32), v[0]);
-      tmem_ld_wait_regs(v[0]);
-    }
+    const int cl = w.col0 + j * 32;   // first column of the chunk within the tile
+    const uint32_t* cur = v[j & 1];
+    if (j + 1 < nch) tmem_ld_32x32b_x32(taddr0 + static_cast<uint32_t>((j + 1) * 32), v[(j + 1) & 1]);
     uint32_t packed[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const float w0 = __shfl_sync(0xffffffffu, sw_lane, 2 * i);
-      const float w1 = __shfl_sync(0xffffffffu, sw_lane, 2 * i + 1);
-      const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i]), sx), w0);
-      const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i + 1]), sx), w1);
+      const float w0 = __shfl_sync(0xffffffffu, pre.sw[j], 2 * i);
+      const float w1 = __shfl_sync(0xffffffffu, pre.sw[j], 2 * i + 1);
+      const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i]), pre.sx), w0);
+      const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i + 1]), pre.sx), w1);
       const __half2 hv = __floats2half2_rn(y0, y1);
       packed[i] = *reinterpret_cast<const uint32_t*>(&hv);
     }
-    // The previous bulk store of this warp must have finished reading the tile.
-    if (lane == 0) bulk_wait_read_all();
+    // The staging tile about to be written must have been read by its last
+    // bulk store (with two tiles: the store of chunk j-2).
+    uint8_t* buf = stage + (kBufs == 2 ? (j & 1) * kEpiWarps * kStageTileBytes : 0);
+    if (lane == 0) {
+      if (kBufs == 2) bulk_wait_read_1();
+      else bulk_wait_read_all();
+    }
     __syncwarp();
+    const uint32_t sbase = smem_u32(buf);
 #pragma unroll
     for (int c = 0; c < 4; ++c)
       st_shared_v4(sbase + stage_off(lane, c), packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-    if (t.tma) {
+    if (bulk) {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_2d(tmY, stage, t.n0 + cl, t.row0 + q * 32);
+        tma_store_2d(tmY, buf, t.n0 + cl, qrow0);
         bulk_commit_group();
       }
     } else {
@@ -161,14 +193,13 @@ __device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams
         const int rr = it * 8 + (lane >> 2);
         const int c = lane & 3;
         const uint4 val = ld_shared_v4(sbase + stage_off(rr, c));
-        const int grow = t.row0 + q * 32 + rr;
         const int gcol = t.n0 + cl + c * 8;
-        if (grow < t.row_end && gcol < p.N)
-          *reinterpret_cast<uint4*>(p.Y + static_cast<int64_t>(grow) * p.N + gcol) = val;
+        if (rr < valid && gcol < p.N)
+          *reinterpret_cast<uint4*>(p.Y + static_cast<int64_t>(qrow0 + rr) * p.N + gcol) = val;
       }
       __syncwarp();
     }
-    if (kDrain && j + 1 < nch) tmem_ld_wait_regs(v[(j + 1) & 1]);
+    if (j + 1 < nch) tmem_ld_wait_regs(v[(j + 1) & 1]);
   }
 }
 

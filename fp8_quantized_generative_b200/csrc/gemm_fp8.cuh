@@ -37,7 +37,8 @@ struct GemmLayout {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kNumBars = 2 * STAGES + 5;   // full, empty, tfull[2], tempty[2], drain
   static constexpr int kTmemCols = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
-  static constexpr int kFixedBytes = STAGES * kStageBytes + kEpiSmemBytes + kNumBars * 8 + 32;
+  static constexpr int kEpiBufs = 1;   // one staging tile per epilogue warp (shared memory goes to the ring)
+  static constexpr int kFixedBytes = STAGES * kStageBytes + epi_smem_bytes(kEpiBufs) + kNumBars * 8 + 32;
   static size_t smem_bytes(int E) { return 1024 + kFixedBytes + 2 * static_cast<size_t>(E + 1) * 4 + 16; }
 };
 
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * L::kABytes;
   uint8_t* sEpi = sB + STAGES * L::kBBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + kEpiSmemBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + epi_smem_bytes(L::kEpiBufs));
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -273,23 +274,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       et.row_end = c.row_end;
       et.n0 = c.n0;
       et.sw0 = c.sw0;
-      // A bulk store clips only at the tensor edge, so it is used unless the
-      // slab crosses into the next expert's rows.
-      et.tma = !kGrouped || c.a_row0 + kBM <= c.row_end;
-      // The CTA's last tile: its epilogue is exposed, so it runs at the drain pace.
-      const bool last_tile = t + static_cast<int>(gridDim.x) >= total;
-      EpiScales<BN / 64> sc{};
-      if (last_tile) sc = epilogue_scales<BN / 64>(et, p, warp, lane, BN);
+      et.clip = !kGrouped;   // dense: rows past the end are past the tensor
+      const EpiWarpView wv = epi_view(et, warp, BN, false);
+      const EpiScales<BN / 64> sc = epilogue_scales<BN / 64>(et, p, wv, lane);
       if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
         raise_error(0x4u);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      if (last_tile)
-        epilogue_slab<BN / 64, true>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, BN, sc);
-      else
-        epilogue_slab<BN / 64, false>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, BN, sc);
+      epilogue_slab<BN / 64, L::kEpiBufs>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), wv, warp, lane,
+                                          stage, sc);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);

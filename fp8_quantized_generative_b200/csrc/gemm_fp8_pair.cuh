@@ -40,7 +40,9 @@ struct PairLayout {
   // per FLOP, but the epilogue no longer overlaps the next tile's MMAs.
   static constexpr bool kWide = BN > 256;
   static constexpr int kNAcc = kWide ? 1 : 2;
-  static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes + kEpiSmemBytes + kNumBars * 8 + 32;
+  static constexpr int kEpiBufs = 2;                   // two staging tiles per epilogue warp
+  static constexpr size_t kSmemBytes =
+      1024 + size_t(STAGES) * kStageBytes + epi_smem_bytes(kEpiBufs) + kNumBars * 8 + 32;
   // plus the MoE schedule tables (offsets and tile prefix) when grouped
   static size_t smem_bytes(int E) { return kSmemBytes + 2 * static_cast<size_t>(E + 1) * 4 + 16; }
 };
@@ -57,6 +59,7 @@ struct PairTile {
   int sw0;      // s_w index of column n0
   int bn;       // width: BN, or BN / tail_q for a tail piece
   bool tail;
+  bool half;    // grouped: M = 128 pair tile (64 rows per CTA) for an expert's last <= 128 rows
 };
 
 template <int BN, bool kGrouped>
@@ -70,16 +73,21 @@ __device__ __forceinline__ PairTile pair_tile(int t, const GemmParams& p, int nu
       if (tile_prefix[mid] <= t) lo = mid; else hi = mid;
     }
     const int e = lo;
-    const int mt = (offs[e + 1] - offs[e] + 2 * kBM - 1) / (2 * kBM);
+    const int cnt = offs[e + 1] - offs[e];
+    const int full = cnt / (2 * kBM);
+    const int rem = cnt - full * 2 * kBM;
+    const int mt = full + (rem > 0 ? 1 : 0);
     const int local = t - tile_prefix[e];
     const int n_blk = local / mt;
-    r.a_row0 = offs[e] + (local - n_blk * mt) * 2 * kBM;
+    const int m_idx = local - n_blk * mt;
+    r.a_row0 = offs[e] + m_idx * 2 * kBM;
     r.row_end = offs[e + 1];
     r.n0 = n_blk * BN;
     r.b_row0 = e * p.N + r.n0;
     r.sw0 = r.b_row0;
     r.bn = BN;
     r.tail = false;
+    r.half = p.half_tiles && m_idx == full && rem <= kBM;
     return r;
   }
   int f, piece = 0;
@@ -99,14 +107,15 @@ __device__ __forceinline__ PairTile pair_tile(int t, const GemmParams& p, int nu
   r.row_end = p.rows;
   r.b_row0 = r.n0;
   r.sw0 = r.n0;
+  r.half = false;
   return r;
 }
 
 template <int BN, int STAGES, bool kGrouped>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmBt, const __grid_constant__ CUtensorMap tmY,
-                         const GemmParams p) {
+    fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAh,
+                         const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBt,
+                         const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
   using L = PairLayout<BN, STAGES>;
   static_assert(BN % 64 == 0 && BN >= 64 && (BN <= 256 || BN == 512) && (BN / 2) % 8 == 0, "BN");
   static_assert(L::kNAcc * BN <= L::kTmemCols, "accumulators must fit in TMEM");
@@ -119,7 +128,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * L::kABytes;
   uint8_t* sEpi = sB + STAGES * L::kBBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + kEpiSmemBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + epi_smem_bytes(L::kEpiBufs));
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -156,6 +165,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
+    if (kGrouped) prefetch_tmap(&tmAh);
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmBt);
     prefetch_tmap(&tmY);
@@ -235,8 +245,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       pdl_wait_prior_grid();
       for (int t = pair; t < total && ok; t += npairs) {
         const PairTile pt = pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs);
-        const int a_row = pt.a_row0 + static_cast<int>(rank) * kBM;
-        const uint32_t bytes = 2u * static_cast<uint32_t>(L::kABytes + (pt.bn / 2) * kBK);
+        // half tile: 64 rows of A per CTA (box of tmAh) at the start of the stage slot
+        const int a_rows = pt.half ? kBM / 2 : kBM;
+        const int a_row = pt.a_row0 + static_cast<int>(rank) * a_rows;
+        const CUtensorMap* tma_a = pt.half ? &tmAh : &tmA;
+        const uint32_t bytes = 2u * static_cast<uint32_t>(a_rows * kBK + (pt.bn / 2) * kBK);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (pre > 0) {
             // stage kb of the first pass: weights already requested
@@ -255,7 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint32_t full_leader = mapa_shared(smem_u32(&full[s]), 0);
           if (leader) mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_2d_pair(sA + s * L::kABytes, &tmA, full_leader, kb * kBK, a_row);
+          tma_load_2d_pair(sA + s * L::kABytes, tma_a, full_leader, kb * kBK, a_row);
           load_b(pt, sB + s * L::kBBytes, full_leader, kb * kBK);
           if (++s == STAGES) {
             s = 0;
@@ -288,7 +301,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
-        const uint32_t idesc = (!kWide && t >= p.main_tiles) ? idesc_e4m3_f32(2 * kBM, BN / p.tail_q) : kIdesc;
+        uint32_t idesc = (!kWide && t >= p.main_tiles) ? idesc_e4m3_f32(2 * kBM, BN / p.tail_q) : kIdesc;
+        // grouped: an M = 128 pair MMA for a half tile (64 rows per CTA)
+        if (kGrouped && pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs).half)
+          idesc = idesc_e4m3_f32(kBM, BN);
         const int halves = kWide ? pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs).bn / 256 : 1;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {
@@ -339,27 +355,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int t = pair; t < total; t += npairs) {
       const PairTile pt = pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs);
       EpiTile et;
-      et.row0 = pt.a_row0 + static_cast<int>(rank) * kBM;
+      et.row0 = pt.a_row0 + static_cast<int>(rank) * (pt.half ? kBM / 2 : kBM);
       et.row_end = pt.row_end;
       et.n0 = pt.n0;
       et.sw0 = pt.sw0;
-      // The bulk store clips only at the tensor edge: used unless this CTA's
-      // slab crosses into the next expert's rows.
-      et.tma = !kGrouped || et.row0 + kBM <= et.row_end;
-      // The CTA's last tile: its epilogue is exposed, so it runs at the drain pace.
-      const bool last_tile = t + static_cast<int>(npairs) >= total;
-      EpiScales<BN / 64> sc{};
-      if (last_tile) sc = epilogue_scales<BN / 64>(et, p, warp, lane, pt.bn);
+      et.clip = !kGrouped;   // dense: rows past the end are past the tensor
+      const EpiWarpView wv = epi_view(et, warp, pt.bn, pt.half);
+      const EpiScales<BN / 64> sc = epilogue_scales<BN / 64>(et, p, wv, lane);
       if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
         raise_error(0x4u);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      if (last_tile)
-        epilogue_slab<BN / 64, true>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, pt.bn, sc);
-      else
-        epilogue_slab<BN / 64, false>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), warp, lane, stage, pt.bn, sc);
+      epilogue_slab<BN / 64, L::kEpiBufs>(et, p, &tmY, tmem_base + static_cast<uint32_t>(acc * BN), wv, warp, lane,
+                                          stage, sc);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);

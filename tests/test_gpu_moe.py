@@ -76,6 +76,9 @@ def test_small_groups_full_compare(fq, family):
     [128, 128, 256],              # exact tile multiples
     [700],                        # E = 1 behaves like a dense linear
     [255, 257, 0, 1, 512, 100],   # 256-row blocks split one row before / after the boundary
+    # CTA-pair kernel: an expert's last 1..128 rows form an M = 128 pair tile
+    # (64 rows per CTA), 129..255 an M = 256 tile; both sides of each edge
+    [64, 65, 127, 128, 129, 191, 320, 383, 384, 385],
 ])
 def test_adversarial_offsets(fq, family, counts):
     E, N, K = len(counts), 256, 256

@@ -10,6 +10,9 @@ any FP32 accumulation order:
     P[m,n] = sum_k dec(Xq[m,k]) * dec(Wq[n,k])          (float64)
     Y[m,n] = fp16_rne( (P[m,n] * s_x[m]) * s_w[n] )     (float64 -> float16)
 
+With activations in E5M2 (['FP8量化在生成式推荐系统OneRec-V2中的优化实践'
+§2.2]) only dec(Xq) changes: x_fmt names the activation codec.
+
 No bias term (the pages name none).  The float64 -> float16 cast is NumPy's
 direct, correctly rounded conversion (round half to even, overflow to inf).
 
@@ -21,18 +24,21 @@ from __future__ import annotations
 import numpy as np
 
 from .e4m3 import e4m3_decode
+from .e5m2 import e5m2_decode
+
+_DECODERS = {"e4m3": e4m3_decode, "e5m2": e5m2_decode}
 
 
-def linear_ref(Xq, s_x, Wq, s_w) -> np.ndarray:
+def linear_ref(Xq, s_x, Wq, s_w, x_fmt: str = "e4m3") -> np.ndarray:
     """Xq uint8 [M,K], s_x f32 [M], Wq uint8 [N,K], s_w f32 [N] -> float16 [M,N]."""
-    Dx = e4m3_decode(Xq)
+    Dx = _DECODERS[x_fmt](Xq)
     Dw = e4m3_decode(Wq)
     P = Dx @ Dw.T
     Y = (P * np.asarray(s_x, dtype=np.float64)[:, None]) * np.asarray(s_w, dtype=np.float64)[None, :]
     return Y.astype(np.float16)
 
 
-def moe_ref(Xq, s_x, offsets, Wq, s_w) -> np.ndarray:
+def moe_ref(Xq, s_x, offsets, Wq, s_w, x_fmt: str = "e4m3") -> np.ndarray:
     """Grouped linear.
 
     Xq uint8 [R,K] (rows in expert order), s_x f32 [R], offsets int [E+1]
@@ -48,7 +54,7 @@ def moe_ref(Xq, s_x, offsets, Wq, s_w) -> np.ndarray:
     for e in range(E):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if hi > lo:
-            Y[lo:hi] = linear_ref(Xq[lo:hi], s_x[lo:hi], Wq[e], s_w[e])
+            Y[lo:hi] = linear_ref(Xq[lo:hi], s_x[lo:hi], Wq[e], s_w[e], x_fmt)
     return Y
 
 

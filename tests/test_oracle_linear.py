@@ -15,7 +15,7 @@ Pins:
 import numpy as np
 import pytest
 
-from oracle import e4m3_decode, linear_f64_unquantized, linear_ref, moe_ref, quant_rows
+from oracle import e4m3_decode, e5m2_decode, linear_f64_unquantized, linear_ref, moe_ref, quant_rows, quant_tensor
 
 
 FINITE_POS = e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))   # 0 .. 448
@@ -144,3 +144,74 @@ def test_moe_rejects_bad_offsets():
     for bad in ([0, 3, 2], [1, 2, 4], [0, 2, 5]):
         with pytest.raises(ValueError):
             moe_ref(Xq, sx, np.array(bad, np.int32), Wq, sw)
+
+
+# ---------------------------------------------------------------------------
+# E5M2 activations ('FP8量化在生成式推荐系统OneRec-V2中的优化实践' §2.2).
+
+E5M2_POS = e5m2_decode(np.arange(0, 0x7C, dtype=np.uint8))    # 0 .. 57344
+
+
+def exact_matrix_e5m2(rng, rows, cols, j):
+    """Entries = random E5M2 value * 2^j; each row holds one ±57344*2^j (fp16-exact for j <= 0)."""
+    v = rng.choice(E5M2_POS[E5M2_POS <= 57344.0], size=(rows, cols)) * rng.choice([-1.0, 1.0], size=(rows, cols))
+    v = np.where(np.abs(v) * 2.0 ** j < 2.0 ** -14, 0.0, v)            # fp16 normals hold every E5M2 value exactly
+    where = rng.integers(0, cols, rows)
+    v[np.arange(rows), where] = 57344.0 * rng.choice([-1.0, 1.0], size=rows)
+    m = (v * 2.0 ** j).astype(np.float16)
+    assert np.all(m.astype(np.float64) == v * 2.0 ** j)
+    return m
+
+
+@pytest.mark.parametrize("M,N,K,jx,jw", [(5, 7, 64, -12, -6), (19, 9, 128, -10, -8)])
+def test_e5m2_exactness_case(M, N, K, jx, jw):
+    rng = np.random.default_rng(M * 77 + N)
+    X = exact_matrix_e5m2(rng, M, K, jx)
+    W = exact_matrix(rng, N, K, jw)
+    Xq, sx = quant_rows(X, "e5m2")
+    Wq, sw = quant_rows(W)
+    assert np.all(sx == np.float32(2.0 ** jx))
+    Y = linear_ref(Xq, sx, Wq, sw, x_fmt="e5m2")
+    expect = (X.astype(np.float64) @ W.astype(np.float64).T).astype(np.float16)
+    np.testing.assert_array_equal(Y.view(np.uint16), expect.view(np.uint16))
+
+
+def quant_error_bound_e5m2(X, W, sx, sw, Y):
+    """As quant_error_bound, with the activation term of a 2-bit mantissa:
+    dx = max(2^-3 |x|, 2^-17 s) (E5M2 half-ulp; subnormal half-step 2^-17)."""
+    xa = np.abs(X.astype(np.float64))
+    wa = np.abs(W.astype(np.float64))
+    dx = np.maximum(2.0 ** -3 * xa, 2.0 ** -17 * sx.astype(np.float64)[:, None]) * (1 + 2.0 ** -18) + xa * 2.0 ** -20
+    dw = np.maximum(2.0 ** -4 * wa, 2.0 ** -10 * sw.astype(np.float64)[:, None]) * (1 + 2.0 ** -18) + wa * 2.0 ** -20
+    prod = (xa + dx) @ (wa + dw).T - xa @ wa.T
+    y = np.abs(Y.astype(np.float64))
+    return prod * (1 + 2.0 ** -40) + 2.0 ** -10 * y + 2.0 ** -24
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_e5m2_brute_force_error_bound(seed):
+    rng = np.random.default_rng(300 + seed)
+    M, N, K = rng.integers(1, 17, 3)
+    X = (rng.standard_normal((M, K)) * np.exp(rng.uniform(-3, 3, (M, 1)))).astype(np.float16)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+    Xq, sx = quant_rows(X, "e5m2")
+    Wq, sw = quant_rows(W)
+    Y = linear_ref(Xq, sx, Wq, sw, x_fmt="e5m2")
+    err = np.abs(Y.astype(np.float64) - linear_f64_unquantized(X, W))
+    assert np.all(err <= quant_error_bound_e5m2(X, W, sx, sw, Y))
+    # decoding the E5M2 codes as E4M3 would be wrong: the bound must catch it
+    wrong = linear_ref(Xq, sx, Wq, sw)
+    finite = np.isfinite(wrong.astype(np.float64))
+    assert np.any(~finite) or np.any(np.abs(wrong.astype(np.float64) - linear_f64_unquantized(X, W))
+                                     > quant_error_bound_e5m2(X, W, sx, sw, wrong))
+
+
+def test_per_tensor_weights_linear_error_bound():
+    rng = np.random.default_rng(51)
+    X = rng.standard_normal((9, 64)).astype(np.float16)
+    W = (rng.standard_normal((12, 64)) * np.linspace(0.005, 0.1, 12)[:, None]).astype(np.float16)
+    Xq, sx = quant_rows(X)
+    Wq, sw = quant_tensor(W)
+    Y = linear_ref(Xq, sx, Wq, sw)
+    err = np.abs(Y.astype(np.float64) - linear_f64_unquantized(X, W))
+    assert np.all(err <= quant_error_bound(X, W, sx, sw, Y))

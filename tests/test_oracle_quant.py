@@ -10,7 +10,7 @@ import os
 import numpy as np
 import pytest
 
-from oracle import EPS, e4m3_decode, quant_rows
+from oracle import EPS, e4m3_decode, e5m2_decode, quant_rows, quant_tensor
 
 
 def _load(golden_dir):
@@ -108,3 +108,103 @@ def test_brute_force_small_rows():
 def test_empty_inputs():
     c, s = quant_rows(np.zeros((0, 16), np.float16))
     assert c.shape == (0, 16) and s.shape == (0,)
+
+
+# ---------------------------------------------------------------------------
+# E5M2 activations ('FP8量化在生成式推荐系统OneRec-V2中的优化实践' §2.2): the same
+# steps with max_code = 57344.
+
+def test_e5m2_hand_worked_rows(golden_dir):
+    with open(os.path.join(golden_dir, "quant_rows_e5m2_hand.json")) as f:
+        cases = json.load(f)["cases"]
+    for case in cases:
+        x = np.array([np.float16(v) for v in case["x"]], dtype=np.float16)[None, :]
+        codes, s = quant_rows(x, "e5m2")
+        exp_codes = np.array([int(c, 16) for c in case["codes"]], dtype=np.uint8)
+        np.testing.assert_array_equal(codes[0], exp_codes, err_msg=case["name"])
+        assert int(s.view(np.uint32)[0]) == int(case["scale_f32_bits"], 16), case["name"]
+
+
+def test_e5m2_row_max_maps_to_57344():
+    rng = np.random.default_rng(33)
+    x = (rng.standard_normal((256, 200)) * np.exp(rng.uniform(-6, 6, (256, 1)))).astype(np.float16)
+    x = x[np.all(np.isfinite(x.astype(np.float32)), axis=1) & (np.abs(x.astype(np.float32)).max(axis=1) > 0)]
+    codes, _ = quant_rows(x, "e5m2")
+    idx = np.argmax(np.abs(x.astype(np.float32)), axis=1)
+    assert np.all((codes[np.arange(len(x)), idx] & 0x7F) == 0x7B)
+
+
+def test_e5m2_dequant_error_bound_per_element():
+    # 2-bit mantissa: |q*s - x| <= max(2^-3 |x|, 2^-17 s) plus fp32 slack.
+    rng = np.random.default_rng(39)
+    x = (rng.standard_normal((64, 512)) * np.exp(rng.uniform(-4, 4, (64, 1)))).astype(np.float16)
+    codes, s = quant_rows(x, "e5m2")
+    deq = e5m2_decode(codes) * s.astype(np.float64)[:, None]
+    xa = np.abs(x.astype(np.float64))
+    bound = np.maximum(2.0 ** -3 * xa, 2.0 ** -17 * s.astype(np.float64)[:, None]) * (1 + 2.0 ** -18) + xa * 2.0 ** -20
+    err = np.abs(deq - x.astype(np.float64))
+    assert np.all(err <= bound)
+    # and the E5M2 error is really coarser than E4M3's on the same rows
+    c4, s4 = quant_rows(x)
+    err4 = np.abs(e4m3_decode(c4) * s4.astype(np.float64)[:, None] - x.astype(np.float64))
+    assert err.mean() > 1.5 * err4.mean()
+
+
+def test_e5m2_brute_force_small_rows():
+    finite = [c for c in range(256) if ((c >> 2) & 0x1F) != 31]
+    table = {c: float(e5m2_decode(np.array([c], np.uint8))[0]) for c in finite}
+    rng = np.random.default_rng(41)
+    x = (rng.standard_normal((5, 40)) * 3).astype(np.float16)
+    codes, s = quant_rows(x, "e5m2")
+    for i in range(x.shape[0]):
+        a = max(float(np.max(np.abs(x[i].astype(np.float32)))), float(EPS))
+        r = np.float32(np.float32(57344.0) / np.float32(a))
+        for k in range(x.shape[1]):
+            t = float(np.float32(np.float32(x[i, k]) * r))
+            t = min(max(t, -57344.0), 57344.0)
+            best = min(finite, key=lambda c: (abs(table[c] - t), c & 1,
+                                              (c >> 7) != (1 if np.signbit(t) else 0)))
+            assert codes[i, k] == best or (t == 0.0 and (codes[i, k] & 0x7F) == 0), (i, k, t)
+
+
+# ---------------------------------------------------------------------------
+# Per-tensor weight scale (same page, §2.1: FFN linears quantized per tensor).
+
+def test_per_tensor_one_scale_and_matches_rows_when_row_maxima_agree():
+    rng = np.random.default_rng(45)
+    w = (rng.standard_normal((24, 96)) * 0.02).astype(np.float16)
+    w[:, 5] = np.float16(0.125)            # every row's amax is 0.125 (all |w| < 0.125 otherwise)
+    w[:, 5][::2] = np.float16(-0.125)
+    assert np.abs(w.astype(np.float32)).max() == np.float32(0.125)
+    codes, s = quant_tensor(w)
+    assert s.shape == (24,) and np.all(s == s[0])
+    c_rows, s_rows = quant_rows(w)
+    np.testing.assert_array_equal(codes, c_rows)
+    np.testing.assert_array_equal(s, s_rows)
+
+
+def test_per_tensor_uses_the_global_maximum():
+    rng = np.random.default_rng(47)
+    w = (rng.standard_normal((16, 64)) * np.linspace(0.01, 1.0, 16)[:, None]).astype(np.float16)
+    codes, s = quant_tensor(w)
+    a = np.float32(np.abs(w.astype(np.float32)).max())
+    assert s[0] == np.float32(a / np.float32(448.0))
+    big = int(np.argmax(np.abs(w.astype(np.float32)).max(axis=1)))
+    # the row holding the global maximum is quantized exactly as by itself
+    c_big, s_big = quant_rows(w[big:big + 1])
+    np.testing.assert_array_equal(codes[big], c_big[0])
+    # other rows use the larger shared scale: every code magnitude <= per-row code magnitude
+    c_rows, _ = quant_rows(w)
+    assert np.all(e4m3_decode(codes & 0x7F) <= e4m3_decode(c_rows & 0x7F))
+    # dequantization error bound with the shared scale
+    deq = e4m3_decode(codes) * np.float64(s[0])
+    wa = np.abs(w.astype(np.float64))
+    bound = np.maximum(2.0 ** -4 * wa, 2.0 ** -10 * np.float64(s[0])) * (1 + 2.0 ** -18) + wa * 2.0 ** -20
+    assert np.all(np.abs(deq - w.astype(np.float64)) <= bound)
+
+
+def test_per_tensor_zero_matrix_and_empty():
+    codes, s = quant_tensor(np.zeros((3, 8), np.float16))
+    assert np.all(codes == 0) and np.all(s == np.float32(EPS / np.float32(448.0)))
+    c, s = quant_tensor(np.zeros((0, 8), np.float16))
+    assert c.shape == (0, 8) and s.shape == (0,)

@@ -139,14 +139,18 @@ class ClockSampler:
 class Plan:
     """Device buffers (rotated sets) and the raw C-ABI launch sequence of one step."""
 
-    def __init__(self, kind, tensors, device, min_rotation_bytes, fused=True):
+    def __init__(self, kind, tensors, device, min_rotation_bytes, fused=True, x_fmt="e4m3", weights="channel"):
         import fp8_quantized_generative_b200 as fq
         from fp8_quantized_generative_b200 import _lib
         self.fq, self.L = fq, _lib
         self.kind = kind
         self.device = device
-        # Up to 16 token rows the library quantizes inside the GEMM (one launch).
-        self.fused = fused and kind == "dense" and tensors[0].shape[0] <= fq.FUSED_MAX_ROWS
+        # activation codes E4M3 (the path) or E5M2 (variant); weight scales per channel or per tensor (variant)
+        self.x_fmt = x_fmt
+        self.weights = weights if kind == "dense" else "channel"   # per-tensor scales: the dense (FFN) variant
+        self.fmt = _lib.FORMATS[x_fmt]
+        # Up to 16 token rows the library quantizes inside the GEMM (one launch; E4M3 only).
+        self.fused = fused and kind == "dense" and x_fmt == "e4m3" and tensors[0].shape[0] <= fq.FUSED_MAX_ROWS
         if kind == "dense":
             X, W = tensors
             self.M, self.K = X.shape
@@ -166,7 +170,8 @@ class Plan:
             b = {}
             if kind == "dense":
                 b["X"] = X.to(device)
-                b["Wq"], b["sw"] = fq.quantize_weight_per_channel(W.to(device))
+                qw = fq.quantize_weight_per_tensor if weights == "tensor" else fq.quantize_weight_per_channel
+                b["Wq"], b["sw"] = qw(W.to(device))
                 b["Xq"] = torch.empty((self.M, self.K), dtype=torch.uint8, device=device)
                 b["sx"] = torch.empty((self.M,), dtype=torch.float32, device=device)
                 b["Y"] = torch.empty((self.M, self.N), dtype=torch.float16, device=device)
@@ -219,20 +224,21 @@ class Plan:
             s = L.fp8q_quantized_linear(p["X"], p["Wq"], p["sw"], self.M, self.N, self.K, p["Y"], 0, 0, st)
         elif self.kind == "dense":
             if k == 0:
-                s = L.fp8q_quantize_rows_dynamic(p["X"], self.M, self.K, p["Xq"], p["sx"], st)
+                s = L.fp8q_quantize_rows_dynamic_fmt(p["X"], self.M, self.K, self.fmt, p["Xq"], p["sx"], st)
             else:
-                s = L.fp8q_linear(p["Xq"], p["sx"], p["Wq"], p["sw"], self.M, self.N, self.K, p["Y"], st)
+                s = L.fp8q_linear_fmt(p["Xq"], self.fmt, p["sx"], p["Wq"], p["sw"], self.M, self.N, self.K, p["Y"],
+                                      st)
         else:
             if k == 0:
-                s = L.fp8q_quantize_rows_dynamic(p["X"], self.R, self.D, p["Xq"], p["sx"], st)
+                s = L.fp8q_quantize_rows_dynamic_fmt(p["X"], self.R, self.D, self.fmt, p["Xq"], p["sx"], st)
             elif k == 1:
-                s = L.fp8q_moe_grouped_linear(p["Xq"], p["sx"], p["off"], self.E, self.R, p["Wuq"], p["swu"],
-                                              self.F, self.D, p["H"], st)
+                s = L.fp8q_moe_grouped_linear_fmt(p["Xq"], self.fmt, p["sx"], p["off"], self.E, self.R, p["Wuq"],
+                                                  p["swu"], self.F, self.D, p["H"], st)
             elif k == 2:
-                s = L.fp8q_quantize_rows_dynamic(p["H"], self.R, self.F, p["Hq"], p["sh"], st)
+                s = L.fp8q_quantize_rows_dynamic_fmt(p["H"], self.R, self.F, self.fmt, p["Hq"], p["sh"], st)
             else:
-                s = L.fp8q_moe_grouped_linear(p["Hq"], p["sh"], p["off"], self.E, self.R, p["Wdq"], p["swd"],
-                                              self.D, self.F, p["Y"], st)
+                s = L.fp8q_moe_grouped_linear_fmt(p["Hq"], self.fmt, p["sh"], p["off"], self.E, self.R, p["Wdq"],
+                                                  p["swd"], self.D, self.F, p["Y"], st)
         if s != 0:
             L.check(s, f"launch {self.kernels[k]}")
 
@@ -352,13 +358,14 @@ def timed_e2e(plan, tensors, steps):
 
 
 # --------------------------------------------------------------------------- oracle arm
-def oracle_sampler(kind, tensors, m_rows, n_rows):
+def oracle_sampler(kind, tensors, m_rows, n_rows, x_fmt="e4m3", weights="channel"):
     """A callable running the oracle on an (m_rows x n_rows) output sample; returns its FLOPs."""
-    from oracle import linear_ref, quant_rows
+    from oracle import linear_ref, quant_rows, quant_tensor
     if kind == "dense":
         X, W = tensors
         Xn = X.numpy()
-        Wq, sw = quant_rows(W.numpy())              # offline weight quantization, untimed
+        # offline weight quantization, untimed
+        Wq, sw = quant_tensor(W.numpy()) if weights == "tensor" else quant_rows(W.numpy())
         K = Xn.shape[1]
         n_rows = min(n_rows, Wq.shape[0])
         m_rows = min(m_rows, Xn.shape[0])
@@ -369,8 +376,8 @@ def oracle_sampler(kind, tensors, m_rows, n_rows):
             state["i"] += 1
             r0 = (i * m_rows) % max(1, Xn.shape[0] - m_rows + 1)
             c0 = (i * n_rows) % max(1, Wq.shape[0] - n_rows + 1)
-            xq, sx = quant_rows(Xn[r0:r0 + m_rows])
-            linear_ref(xq, sx, Wq[c0:c0 + n_rows], sw[c0:c0 + n_rows])
+            xq, sx = quant_rows(Xn[r0:r0 + m_rows], x_fmt)
+            linear_ref(xq, sx, Wq[c0:c0 + n_rows], sw[c0:c0 + n_rows], x_fmt)
             return 2.0 * m_rows * n_rows * K
         return run, f"{m_rows} activation rows x {n_rows} weight rows (output block) per call"
     Xp, offsets, Wu, Wd = tensors
@@ -383,11 +390,11 @@ def oracle_sampler(kind, tensors, m_rows, n_rows):
     D = Xn.shape[1]
 
     def run():
-        xq, sx = quant_rows(Xn)
-        h = linear_ref(xq, sx, Wuq, swu)
-        hq, sh = quant_rows(h)
+        xq, sx = quant_rows(Xn, x_fmt)
+        h = linear_ref(xq, sx, Wuq, swu, x_fmt)
+        hq, sh = quant_rows(h, x_fmt)
         # down projection restricted to the sampled hidden columns
-        linear_ref(hq, sh, Wdq[:n_rows, :hq.shape[1]], swd[:n_rows])
+        linear_ref(hq, sh, Wdq[:n_rows, :hq.shape[1]], swd[:n_rows], x_fmt)
         return 2.0 * cnt * Wuq.shape[0] * D + 2.0 * cnt * n_rows * hq.shape[1]
     return run, f"expert {e}: {cnt} rows through up ({n_rows} channels) and down ({n_rows} channels)"
 
@@ -403,8 +410,8 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def cpu_baseline(kind, tensors, budget_s=10.0):
-    run, sample = oracle_sampler(kind, tensors, 64, 6144 if kind == "dense" else 1024)
+def cpu_baseline(kind, tensors, budget_s=10.0, x_fmt="e4m3", weights="channel"):
+    run, sample = oracle_sampler(kind, tensors, 64, 6144 if kind == "dense" else 1024, x_fmt, weights)
     run()                                           # warm (page-in, BLAS threads)
     flops, t0 = 0.0, time.perf_counter()
     while True:
@@ -459,7 +466,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     desc, kind, tensors = workload_spec(args.workload)
-    run, sample = oracle_sampler(kind, tensors, 32, 256)
+    run, sample = oracle_sampler(kind, tensors, 32, 256, args.x_fmt, args.weight_scales)
     for _ in range(args.warmup):
         run()
     flops, t0 = 0.0, time.perf_counter()
@@ -471,7 +478,9 @@ def run_reference(args, world, rank):
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": desc, "sample_per_step": sample, "parallelism": "host cores (rank 0 only)"},
+            "config": {"workload": desc, "sample_per_step": sample, "parallelism": "host cores (rank 0 only)",
+                       "activation_format": args.x_fmt,
+                       "weight_scales": "per-" + (args.weight_scales if kind == "dense" else "channel")},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -486,7 +495,8 @@ def run_ours(args, world, rank, local):
     desc, kind, tensors = workload_spec(args.workload)
     import fp8_quantized_generative_b200 as fq
     fq.set_gemm_tuning({"auto": 0, "single": 1, "pair": 2, "splitk": 3}[args.gemm], args.bn, args.ksplit)
-    plan = Plan(kind, tensors, device, min_rotation_bytes=3 * L2_BYTES, fused=args.fused)
+    plan = Plan(kind, tensors, device, min_rotation_bytes=3 * L2_BYTES, fused=args.fused, x_fmt=args.x_fmt,
+                weights=args.weight_scales)
     peaks, peak_src = load_peaks()
 
     sampler = ClockSampler(local)
@@ -545,10 +555,13 @@ def run_ours(args, world, rank, local):
     ms_step = t_max_ms / args.steps
     return {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3 (fp32 accumulate, fp16 out)",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": ("fp8e4m3" if args.x_fmt == "e4m3" else "fp8 e5m2 activations x e4m3 weights")
+                     + " (fp32 accumulate, fp16 out)",
             "data": "synthetic",
             "config": {"workload": desc, "parallelism": f"replicas x{world} (no collective)",
                        "gemm": args.gemm, "bn": args.bn, "ksplit": args.ksplit,
+                       "activation_format": args.x_fmt, "weight_scales": "per-" + plan.weights,
                        "l2": f"rotating {plan.sets} buffer sets of {plan.bytes_per_set / 1e6:.0f} MB "
                              f"(> 3x 126 MB L2), no flush",
                        "step": " -> ".join(plan.kernels),
@@ -604,6 +617,10 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of a CUDA graph")
+    ap.add_argument("--x-fmt", default="e4m3", choices=["e4m3", "e5m2"],
+                    help="activation code format (e5m2: the pages' activation-format variant)")
+    ap.add_argument("--weight-scales", default="channel", choices=["channel", "tensor"],
+                    help="weight scale granularity for dense workloads (tensor: the pages' FFN variant)")
     ap.add_argument("--fused", action="store_true",
                     help="one fused quantize+linear launch per step where it applies (<= 16 rows); "
                          "default: the two launches, measured faster on B200")
@@ -628,7 +645,7 @@ def main(argv=None):
         if rank == 0 and out is not None:
             if world == 1 and not args.no_cpu_baseline:
                 _, kind, tensors = workload_spec(args.workload)
-                out["cpu_baseline"] = cpu_baseline(kind, tensors)
+                out["cpu_baseline"] = cpu_baseline(kind, tensors, x_fmt=args.x_fmt, weights=args.weight_scales)
             else:
                 out["cpu_baseline"] = None
     if rank == 0 and out is not None:

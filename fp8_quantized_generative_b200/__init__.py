@@ -11,6 +11,10 @@ missing library raises ImportError at the first call.
     Wq, s_w = quantize_weight_per_channel(W)    # offline, W fp16 [N,K]
     Y = linear(Xq, s_x, Wq, s_w)                # fp16 [M,N]
     Y = moe_grouped_linear(Xq, s_x, offsets, Wq_e, s_w_e)
+
+Variants from the pages: activations in E5M2 (quantize_rows_dynamic(X,
+fmt="e5m2") with linear(..., x_fmt="e5m2")) and per-tensor weight scales
+(quantize_weight_per_tensor).
 """
 from __future__ import annotations
 
@@ -20,9 +24,16 @@ from . import _lib
 from ._lib import Fp8qError, check, lib
 
 __all__ = [
-    "Fp8qError", "lib", "quantize_rows_dynamic", "quantize_weight_per_channel", "linear",
-    "moe_grouped_linear", "quantized_linear", "e4m3_encode_f32", "device_error", "set_gemm_tuning",
+    "Fp8qError", "lib", "quantize_rows_dynamic", "quantize_weight_per_channel", "quantize_weight_per_tensor",
+    "linear", "moe_grouped_linear", "quantized_linear", "e4m3_encode_f32", "device_error", "set_gemm_tuning",
 ]
+
+
+def _fmt(name: str) -> int:
+    try:
+        return _lib.FORMATS[name]
+    except KeyError:
+        raise ValueError(f"unknown FP8 format {name!r} (e4m3 or e5m2)") from None
 
 
 def _stream(t: torch.Tensor) -> int:
@@ -42,15 +53,20 @@ def _need(t: torch.Tensor, dtype, name: str, ndim: int | None = None):
         raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
 
 
-def quantize_rows_dynamic(X: torch.Tensor, out: tuple | None = None):
-    """Per-token dynamic E4M3 quantization: fp16 [M,K] -> (uint8 [M,K], fp32 [M])."""
+def quantize_rows_dynamic(X: torch.Tensor, out: tuple | None = None, fmt: str = "e4m3"):
+    """Per-token dynamic FP8 quantization: fp16 [M,K] -> (uint8 [M,K], fp32 [M]).
+    fmt: "e4m3" (the path) or "e5m2" (the activation-format variant)."""
     _need(X, torch.float16, "X", 2)
     M, K = X.shape
     Xq, s = out if out is not None else (
         torch.empty((M, K), dtype=torch.uint8, device=X.device),
         torch.empty((M,), dtype=torch.float32, device=X.device))
-    check(_lib.fp8q_quantize_rows_dynamic(X.data_ptr(), M, K, Xq.data_ptr(), s.data_ptr(), _stream(X)),
-          "fp8q_quantize_rows_dynamic")
+    if fmt == "e4m3":
+        check(_lib.fp8q_quantize_rows_dynamic(X.data_ptr(), M, K, Xq.data_ptr(), s.data_ptr(), _stream(X)),
+              "fp8q_quantize_rows_dynamic")
+    else:
+        check(_lib.fp8q_quantize_rows_dynamic_fmt(X.data_ptr(), M, K, _fmt(fmt), Xq.data_ptr(), s.data_ptr(),
+                                                  _stream(X)), "fp8q_quantize_rows_dynamic_fmt")
     return Xq, s
 
 
@@ -68,9 +84,22 @@ def quantize_weight_per_channel(W: torch.Tensor):
     return Wq, s
 
 
+def quantize_weight_per_tensor(W: torch.Tensor):
+    """Offline per-tensor E4M3 quantization of fp16 [N,K]: one scale for the
+    matrix, returned replicated as fp32 [N] (the form linear() takes)."""
+    _need(W, torch.float16, "W", 2)
+    N, K = W.shape
+    Wq = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    s = torch.empty((N,), dtype=torch.float32, device=W.device)
+    check(_lib.fp8q_quantize_weight_per_tensor(W.data_ptr(), N, K, Wq.data_ptr(), s.data_ptr(), _stream(W)),
+          "fp8q_quantize_weight_per_tensor")
+    return Wq, s
+
+
 def linear(Xq: torch.Tensor, s_x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
-           out: torch.Tensor | None = None) -> torch.Tensor:
-    """FP8 W8A8 linear with fused dequantization: fp16 [M,N]."""
+           out: torch.Tensor | None = None, x_fmt: str = "e4m3") -> torch.Tensor:
+    """FP8 W8A8 linear with fused dequantization: fp16 [M,N].  x_fmt: the
+    format of the activation codes Xq ("e4m3" or "e5m2"); weights are E4M3."""
     _need(Xq, torch.uint8, "Xq", 2)
     _need(Wq, torch.uint8, "Wq", 2)
     _need(s_x, torch.float32, "s_x", 1)
@@ -80,8 +109,12 @@ def linear(Xq: torch.Tensor, s_x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Ten
     if Wq.shape[1] != K or s_x.shape[0] != M or s_w.shape[0] != N:
         raise ValueError("shape mismatch")
     Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=Xq.device)
-    check(_lib.fp8q_linear(Xq.data_ptr(), s_x.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K, Y.data_ptr(),
-                           _stream(Xq)), "fp8q_linear")
+    if x_fmt == "e4m3":
+        check(_lib.fp8q_linear(Xq.data_ptr(), s_x.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K, Y.data_ptr(),
+                               _stream(Xq)), "fp8q_linear")
+    else:
+        check(_lib.fp8q_linear_fmt(Xq.data_ptr(), _fmt(x_fmt), s_x.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K,
+                                   Y.data_ptr(), _stream(Xq)), "fp8q_linear_fmt")
     return Y
 
 
@@ -114,8 +147,9 @@ def quantized_linear(X: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
 
 
 def moe_grouped_linear(Xq: torch.Tensor, s_x: torch.Tensor, offsets: torch.Tensor, Wq: torch.Tensor,
-                       s_w: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
-    """Expert-grouped FP8 linear.  offsets: int32 [E+1] on the device."""
+                       s_w: torch.Tensor, out: torch.Tensor | None = None, x_fmt: str = "e4m3") -> torch.Tensor:
+    """Expert-grouped FP8 linear.  offsets: int32 [E+1] on the device; x_fmt
+    the format of the activation codes ("e4m3" or "e5m2")."""
     _need(Xq, torch.uint8, "Xq", 2)
     _need(s_x, torch.float32, "s_x", 1)
     _need(offsets, torch.int32, "offsets", 1)
@@ -126,9 +160,14 @@ def moe_grouped_linear(Xq: torch.Tensor, s_x: torch.Tensor, offsets: torch.Tenso
     if K2 != K or offsets.shape[0] != E + 1 or tuple(s_w.shape) != (E, N) or s_x.shape[0] != rows:
         raise ValueError("shape mismatch")
     Y = out if out is not None else torch.empty((rows, N), dtype=torch.float16, device=Xq.device)
-    check(_lib.fp8q_moe_grouped_linear(Xq.data_ptr(), s_x.data_ptr(), offsets.data_ptr(), E, rows, Wq.data_ptr(),
-                                       s_w.data_ptr(), N, K, Y.data_ptr(), _stream(Xq)),
-          "fp8q_moe_grouped_linear")
+    if x_fmt == "e4m3":
+        check(_lib.fp8q_moe_grouped_linear(Xq.data_ptr(), s_x.data_ptr(), offsets.data_ptr(), E, rows, Wq.data_ptr(),
+                                           s_w.data_ptr(), N, K, Y.data_ptr(), _stream(Xq)),
+              "fp8q_moe_grouped_linear")
+    else:
+        check(_lib.fp8q_moe_grouped_linear_fmt(Xq.data_ptr(), _fmt(x_fmt), s_x.data_ptr(), offsets.data_ptr(), E, rows,
+                                               Wq.data_ptr(), s_w.data_ptr(), N, K, Y.data_ptr(), _stream(Xq)),
+              "fp8q_moe_grouped_linear_fmt")
     return Y
 
 

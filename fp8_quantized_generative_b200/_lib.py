@@ -19,6 +19,10 @@ FP8Q_ERR_CUDA = 3
 FP8Q_ERR_TIMEOUT = 4
 FP8Q_ERR_DEVICE_CHECK = 5
 
+FP8Q_FMT_E4M3 = 0
+FP8Q_FMT_E5M2 = 1
+FORMATS = {"e4m3": FP8Q_FMT_E4M3, "e5m2": FP8Q_FMT_E5M2}
+
 DEVERR_TIMEOUT_PRODUCER = 0x1
 DEVERR_TIMEOUT_MMA = 0x2
 DEVERR_TIMEOUT_EPILOGUE = 0x4
@@ -49,6 +53,10 @@ SIGNATURES = {
     "fp8q_moe_grouped_linear": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_quantized_linear": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P]),
     "fp8q_quantized_linear_noalloc": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "fp8q_quantize_rows_dynamic_fmt": (_INT, [_P, _I64, _I64, _INT, _P, _P, _P]),
+    "fp8q_quantize_weight_per_tensor": (_INT, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8q_linear_fmt": (_INT, [_P, _INT, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "fp8q_moe_grouped_linear_fmt": (_INT, [_P, _INT, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_e4m3_encode_f32": (_INT, [_P, _I64, _P, _P]),
     "fp8q_set_gemm_tuning": (_INT, [_INT, _INT, _INT]),
     "fp8q_selftest_wait_timeout": (_INT, [ctypes.c_uint32, _P]),
@@ -114,6 +122,22 @@ def fp8q_quantized_linear_noalloc(X, Wq, s_w, M, N, K, Y, stream):
 
 def fp8q_moe_grouped_linear(Xq, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream):
     return lib().fp8q_moe_grouped_linear(Xq, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream)
+
+
+def fp8q_quantize_rows_dynamic_fmt(X, M, K, fmt, Xq, s_x, stream):
+    return lib().fp8q_quantize_rows_dynamic_fmt(X, M, K, fmt, Xq, s_x, stream)
+
+
+def fp8q_quantize_weight_per_tensor(W, N, K, Wq, s_w, stream):
+    return lib().fp8q_quantize_weight_per_tensor(W, N, K, Wq, s_w, stream)
+
+
+def fp8q_linear_fmt(Xq, x_fmt, s_x, Wq, s_w, M, N, K, Y, stream):
+    return lib().fp8q_linear_fmt(Xq, x_fmt, s_x, Wq, s_w, M, N, K, Y, stream)
+
+
+def fp8q_moe_grouped_linear_fmt(Xq, x_fmt, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream):
+    return lib().fp8q_moe_grouped_linear_fmt(Xq, x_fmt, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream)
 
 
 def fp8q_e4m3_encode_f32(x, n, out, stream):

@@ -542,13 +542,46 @@ fp8q_status check_quant_args(const void* X, int64_t M, int64_t K, const void* Q,
   return FP8Q_OK;
 }
 
-fp8q_status quantize(const void* X, int64_t M, int64_t K, uint8_t* Q, float* S, void* stream) {
+bool valid_fmt(int fmt) { return fmt == FP8Q_FMT_E4M3 || fmt == FP8Q_FMT_E5M2; }
+
+fp8q_status quantize(const void* X, int64_t M, int64_t K, uint8_t* Q, float* S, void* stream,
+                     int fmt = FP8Q_FMT_E4M3) {
   fp8q_status s = check_quant_args(X, M, K, Q, S);
   if (s != FP8Q_OK || M == 0) return s;
-  const cudaError_t e = launch_quant_rows(static_cast<const __half*>(X), static_cast<int>(M), static_cast<int>(K),
-                                          Q, S, static_cast<cudaStream_t>(stream));
+  const __half* Xh = static_cast<const __half*>(X);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = fmt == FP8Q_FMT_E5M2
+                            ? launch_quant_rows<kFmtE5M2>(Xh, static_cast<int>(M), static_cast<int>(K), Q, S, st)
+                            : launch_quant_rows<kFmtE4M3>(Xh, static_cast<int>(M), static_cast<int>(K), Q, S, st);
   if (e != cudaSuccess) return cuda_fail(e, "quant_rows launch");
   return FP8Q_OK;
+}
+
+// Dense linear, activations in format x_fmt (weights E4M3).
+fp8q_status linear_impl(const uint8_t* Xq, int x_fmt, const float* s_x, const uint8_t* Wq, const float* s_w,
+                        int64_t M, int64_t N, int64_t K, void* Y_f16, void* stream) {
+  if (!valid_fmt(x_fmt)) return invalid("x_fmt must be FP8Q_FMT_E4M3 or FP8Q_FMT_E5M2");
+  if (M < 0 || M > kMaxDim) return invalid("M out of range");
+  if (N <= 0 || N > kMaxDim || N % 8 != 0) return invalid("N must be positive and a multiple of 8");
+  if (K <= 0 || K > kMaxDim || K % 16 != 0) return invalid("K must be positive and a multiple of 16");
+  if (M == 0) return FP8Q_OK;
+  if (!aligned16(Xq) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y_f16))
+    return invalid("null or non-16-byte-aligned pointer");
+  GemmParams p = {};   // every field set below; zero for the rest
+  p.s_x = s_x;
+  p.s_w = s_w;
+  p.Y = static_cast<__half*>(Y_f16);
+  p.offsets = nullptr;
+  p.rows = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.E = 1;
+  p.n_fastest = 0;
+  p.main_tiles = 0;
+  p.tail_q = 1;
+  p.l2_prefetch = l2_prefetch_enabled();
+  p.x_fmt = x_fmt;
+  return launch_dense(Xq, Wq, p, static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -619,28 +652,43 @@ fp8q_status fp8q_quantize_weight_per_channel(const void* W_f16, int64_t N, int64
   return quantize(W_f16, N, K, Wq, s_w, stream);
 }
 
+fp8q_status fp8q_quantize_rows_dynamic_fmt(const void* X_f16, int64_t M, int64_t K, fp8q_format fmt, uint8_t* Xq,
+                                           float* s_x, void* stream) {
+  if (!valid_fmt(fmt)) return invalid("fmt must be FP8Q_FMT_E4M3 or FP8Q_FMT_E5M2");
+  return quantize(X_f16, M, K, Xq, s_x, stream, fmt);
+}
+
+fp8q_status fp8q_quantize_weight_per_tensor(const void* W_f16, int64_t N, int64_t K, uint8_t* Wq, float* s_w,
+                                            void* stream) {
+  if (N == 0) return invalid("N must be positive");
+  fp8q_status s = check_quant_args(W_f16, N, K, Wq, s_w);
+  if (s != FP8Q_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __half* W = static_cast<const __half*>(W_f16);
+  const int64_t nvec = N * K / 8;
+  int dev = 0, sms = 0;
+  cudaError_t e = current_device_info(&dev, &sms);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  const int64_t want = (nvec + 255) / 256;
+  const int grid = static_cast<int>(want < 4 * sms ? want : 4 * sms);
+  e = cudaMemsetAsync(s_w, 0, sizeof(float), st);   // S[0] accumulates the amax bits
+  if (e == cudaSuccess)
+    e = launch_pdl(tensor_amax_kernel, dim3(grid), dim3(256), st, W, nvec, reinterpret_cast<unsigned int*>(s_w));
+  if (e == cudaSuccess)
+    e = launch_pdl(quant_tensor_kernel, dim3(grid), dim3(256), st, W, static_cast<int>(N), nvec, Wq, s_w);
+  if (e == cudaSuccess) e = launch_pdl(quant_tensor_finish_kernel, dim3(1), dim3(32), st, s_w);
+  if (e != cudaSuccess) return cuda_fail(e, "per-tensor quantization launch");
+  return FP8Q_OK;
+}
+
 fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, const float* s_w, int64_t M,
                         int64_t N, int64_t K, void* Y_f16, void* stream) {
-  if (M < 0 || M > kMaxDim) return invalid("M out of range");
-  if (N <= 0 || N > kMaxDim || N % 8 != 0) return invalid("N must be positive and a multiple of 8");
-  if (K <= 0 || K > kMaxDim || K % 16 != 0) return invalid("K must be positive and a multiple of 16");
-  if (M == 0) return FP8Q_OK;
-  if (!aligned16(Xq) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y_f16))
-    return invalid("null or non-16-byte-aligned pointer");
-  GemmParams p = {};   // every field set below; zero for the rest
-  p.s_x = s_x;
-  p.s_w = s_w;
-  p.Y = static_cast<__half*>(Y_f16);
-  p.offsets = nullptr;
-  p.rows = static_cast<int>(M);
-  p.N = static_cast<int>(N);
-  p.K = static_cast<int>(K);
-  p.E = 1;
-  p.n_fastest = 0;
-  p.main_tiles = 0;
-  p.tail_q = 1;
-  p.l2_prefetch = l2_prefetch_enabled();
-  return launch_dense(Xq, Wq, p, static_cast<cudaStream_t>(stream));
+  return linear_impl(Xq, FP8Q_FMT_E4M3, s_x, Wq, s_w, M, N, K, Y_f16, stream);
+}
+
+fp8q_status fp8q_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, const float* s_x, const uint8_t* Wq,
+                            const float* s_w, int64_t M, int64_t N, int64_t K, void* Y_f16, void* stream) {
+  return linear_impl(Xq, x_fmt, s_x, Wq, s_w, M, N, K, Y_f16, stream);
 }
 
 fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const float* s_w, int64_t M, int64_t N,
@@ -704,6 +752,13 @@ fp8q_status fp8q_quantized_linear_noalloc(const void* X_f16, const uint8_t* Wq, 
 fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const int32_t* offsets, int32_t E,
                                     int64_t rows, const uint8_t* Wq, const float* s_w, int64_t N, int64_t K,
                                     void* Y_f16, void* stream) {
+  return fp8q_moe_grouped_linear_fmt(Xq, FP8Q_FMT_E4M3, s_x, offsets, E, rows, Wq, s_w, N, K, Y_f16, stream);
+}
+
+fp8q_status fp8q_moe_grouped_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, const float* s_x,
+                                        const int32_t* offsets, int32_t E, int64_t rows, const uint8_t* Wq,
+                                        const float* s_w, int64_t N, int64_t K, void* Y_f16, void* stream) {
+  if (!valid_fmt(x_fmt)) return invalid("x_fmt must be FP8Q_FMT_E4M3 or FP8Q_FMT_E5M2");
   if (E < 1 || E > kMaxExperts) return invalid("E must be in [1, 1024]");
   if (rows < 0 || rows > kMaxDim) return invalid("rows out of range");
   if (N <= 0 || N % 8 != 0 || int64_t(E) * N > kMaxDim) return invalid("N must be positive, a multiple of 8, E*N < 2^31");
@@ -726,6 +781,7 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x, const i
   p.tail_q = 1;
   p.l2_prefetch = l2_prefetch_enabled();
   p.half_tiles = knobs().half_tiles;
+  p.x_fmt = x_fmt;
   // Single-CTA 128-row tiles by default; kernel family 2 selects CTA-pair
   // tiles of 256 expert rows (each weight tile read by half as many row
   // blocks), which measured no faster for the up projection and slower for

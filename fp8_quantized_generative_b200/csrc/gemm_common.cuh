@@ -44,6 +44,7 @@ struct GemmParams {
   int tail_q;
   int l2_prefetch;          // split-K: 1 = prefetch the rest of the weight slice into L2 at start
   int half_tiles;           // CTA-pair grouped kernel: an expert's last <= 128 rows as an M = 128 pair tile
+  int x_fmt;                // activation code format (Fp8Fmt): E4M3, or E5M2 for the variant
 };
 
 // One output slab of a CTA: 128 rows starting at row0, BN columns at n0.

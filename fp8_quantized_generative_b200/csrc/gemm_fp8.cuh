@@ -96,7 +96,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
   using L = GemmLayout<BN, STAGES>;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
-  constexpr uint32_t kIdesc = idesc_e4m3_f32(kBM, BN);
+  // A = activations: E4M3, or E5M2 for the activation-format variant
+  const uint32_t kIdesc = idesc_e4m3_f32(kBM, BN) | idesc_a_fmt(p.x_fmt);
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);

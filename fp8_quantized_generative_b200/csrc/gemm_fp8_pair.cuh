@@ -120,7 +120,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(BN % 64 == 0 && BN >= 64 && (BN <= 256 || BN == 512) && (BN / 2) % 8 == 0, "BN");
   static_assert(L::kNAcc * BN <= L::kTmemCols, "accumulators must fit in TMEM");
   constexpr bool kWide = L::kWide;
-  constexpr uint32_t kIdesc = idesc_e4m3_f32(2 * kBM, kWide ? 256 : BN);
+  // A = activations: E4M3, or E5M2 for the activation-format variant
+  const uint32_t kAFmt = idesc_a_fmt(p.x_fmt);
+  const uint32_t kIdesc = idesc_e4m3_f32(2 * kBM, kWide ? 256 : BN) | kAFmt;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -301,10 +303,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
-        uint32_t idesc = (!kWide && t >= p.main_tiles) ? idesc_e4m3_f32(2 * kBM, BN / p.tail_q) : kIdesc;
+        uint32_t idesc = (!kWide && t >= p.main_tiles) ? idesc_e4m3_f32(2 * kBM, BN / p.tail_q) | kAFmt : kIdesc;
         // grouped: an M = 128 pair MMA for a half tile (64 rows per CTA)
         if (kGrouped && pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs).half)
-          idesc = idesc_e4m3_f32(kBM, BN);
+          idesc = idesc_e4m3_f32(kBM, BN) | kAFmt;
         const int halves = kWide ? pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs).bn / 256 : 1;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {

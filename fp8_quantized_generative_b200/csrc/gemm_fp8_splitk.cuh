@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
                            const GemmParams p) {
   using L = SplitKLayout<MPAD, STAGES>;
   static_assert(MPAD % 16 == 0 && MPAD >= 16 && MPAD <= 128, "MPAD");
-  constexpr uint32_t kIdesc = idesc_e4m3_f32(kBM, MPAD);
+  // swap-AB: B = activations (E4M3, or E5M2 for the variant; the fused path is E4M3)
+  const uint32_t kIdesc = idesc_e4m3_f32(kBM, MPAD) | idesc_b_fmt(kFused ? kFmtE4M3 : p.x_fmt);
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);

@@ -191,12 +191,16 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
 }
 
 // Instruction descriptor for kind::f8f6f4, E4M3 x E4M3 -> F32, both operands
-// K-major, dense: D format bits 4-5 (1 = F32), A format bits 7-9 (0 = E4M3),
-// B format bits 10-12 (0 = E4M3), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+// K-major, dense: D format bits 4-5 (1 = F32), A format bits 7-9 (0 = E4M3,
+// 1 = E5M2), B format bits 10-12 (same codes), N >> 3 in bits 17-22, M >> 4
+// in bits 24-28.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {
   return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
 }
+// Operand-format fields to OR into a descriptor for an A or B operand in format f.
+__host__ __device__ constexpr uint32_t idesc_a_fmt(int f) { return static_cast<uint32_t>(f) << 7; }
+__host__ __device__ constexpr uint32_t idesc_b_fmt(int f) { return static_cast<uint32_t>(f) << 10; }
 
 // ---------------------------------------------------------------- E4M3 cast
 // Two fp32 -> two E4M3 codes, round to nearest even, saturating to ±448
@@ -204,6 +208,22 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {
 // Returns lo | hi << 8.
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+// The same for E5M2 (cvt.rn.satfinite.e5m2x2.f32): saturates to ±57344.
+__device__ __forceinline__ uint16_t cvt_e5m2x2(float lo, float hi) {
+  return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E5M2));
+}
+
+// FP8 code formats of the path: weights always E4M3; activations E4M3 or,
+// as a variant, E5M2.  The values double as the tcgen05 kind::f8f6f4
+// operand-format field of the instruction descriptor.
+enum Fp8Fmt : int { kFmtE4M3 = 0, kFmtE5M2 = 1 };
+
+template <int F>
+__device__ __forceinline__ uint16_t cvt_fp8x2(float lo, float hi) {
+  static_assert(F == kFmtE4M3 || F == kFmtE5M2, "format");
+  return F == kFmtE4M3 ? cvt_e4m3x2(lo, hi) : cvt_e5m2x2(lo, hi);
 }
 
 }  // namespace fp8q

@@ -1,10 +1,12 @@
-// Per-row dynamic E4M3 quantization (per-token activations at run time,
+// Per-row dynamic FP8 quantization (per-token activations at run time,
 // per-output-channel weights offline).  HBM-bound: 2 bytes read and 1 byte
 // written per element plus 4 bytes of scale per row.
 //
 // Method: "Quantized Inference for OneRec-V2" (关键证据, steps 1-2) and
 // "FP8量化在生成式推荐系统OneRec-V2中的优化实践" §2.2 (scale = max_code / max(|x|, eps)),
-// with max_code = 448, the E4M3 maximum (§1.2).
+// with max_code = 448, the E4M3 maximum (§1.2), or 57344 for the E5M2
+// activation variant (same page, §2.2).  Per-tensor variant (same page, §2.1,
+// FFN weights): one amax over the whole matrix, at the end of this file.
 //
 // Design: a row is held in registers by TPR threads (TPR in {32..256}), each
 // loading VPT 16-byte vectors (8 fp16 values) with coalesced 128-bit loads;
@@ -19,18 +21,25 @@
 namespace fp8q {
 
 constexpr float kE4M3Max = 448.0f;
+constexpr float kE5M2Max = 57344.0f;
 constexpr float kScaleEps = 1e-12f;
 
+template <int F>
+__host__ __device__ constexpr float fp8_max() {
+  return F == kFmtE4M3 ? kE4M3Max : kE5M2Max;
+}
+
 struct RowScale {
-  float r;  // 448 / a'   (multiplier that maps the row max onto 448)
-  float s;  // a' / 448   (stored dequantization scale)
+  float r;  // max_code / a'   (multiplier that maps the row max onto max_code)
+  float s;  // a' / max_code   (stored dequantization scale)
 };
 
+template <int F = kFmtE4M3>
 __device__ __forceinline__ RowScale row_scale_from_amax(float amax) {
   const float a = fmaxf(amax, kScaleEps);
   RowScale rs;
-  rs.r = __fdiv_rn(kE4M3Max, a);
-  rs.s = __fdiv_rn(a, kE4M3Max);
+  rs.r = __fdiv_rn(fp8_max<F>(), a);
+  rs.s = __fdiv_rn(a, fp8_max<F>());
   return rs;
 }
 
@@ -44,20 +53,21 @@ __device__ __forceinline__ float absmax8(const uint4& v, float m) {
   return m;
 }
 
-// 8 fp16 -> 8 E4M3 codes (one fp32 multiply by r each, RN), packed little-endian.
+// 8 fp16 -> 8 FP8 codes (one fp32 multiply by r each, RN), packed little-endian.
+template <int F = kFmtE4M3>
 __device__ __forceinline__ uint2 encode8(const uint4& v, float r) {
   const __half2* h = reinterpret_cast<const __half2*>(&v);
   uint32_t w[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float2 f = __half22float2(h[i]);
-    w[i] = cvt_e4m3x2(__fmul_rn(f.x, r), __fmul_rn(f.y, r));
+    w[i] = cvt_fp8x2<F>(__fmul_rn(f.x, r), __fmul_rn(f.y, r));
   }
   return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
 // Grid: ceil(M / (256 / TPR)) CTAs of 256 threads; TPR threads per row.
-template <int TPR, int VPT>
+template <int TPR, int VPT, int F>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const __half* __restrict__ X, int M, int K,
                                                         uint8_t* __restrict__ Q, float* __restrict__ S) {
   static_assert(TPR >= 32 && TPR <= 256 && (TPR & (TPR - 1)) == 0, "TPR");
@@ -101,17 +111,18 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __half* __restric
   }
   if (!live) return;
 
-  const RowScale rs = row_scale_from_amax(m);
+  const RowScale rs = row_scale_from_amax<F>(m);
   uint2* dst = reinterpret_cast<uint2*>(Q + static_cast<int64_t>(row) * K);
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int j = t + i * TPR;
-    if (j < nvec) dst[j] = encode8(v[i], rs.r);
+    if (j < nvec) dst[j] = encode8<F>(v[i], rs.r);
   }
   if (t == 0) S[row] = rs.s;
 }
 
 // Any K (multiple of 8): one CTA of 256 threads per row, two passes over the row.
+template <int F>
 __global__ void __launch_bounds__(256) quant_rows_long_kernel(const __half* __restrict__ X, int M, int K,
                                                              uint8_t* __restrict__ Q, float* __restrict__ S) {
   __shared__ float red[8];
@@ -128,10 +139,64 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const __half* __re
   __syncthreads();
 #pragma unroll
   for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
-  const RowScale rs = row_scale_from_amax(m);
+  const RowScale rs = row_scale_from_amax<F>(m);
   uint2* dst = reinterpret_cast<uint2*>(Q + static_cast<int64_t>(row) * K);
-  for (int j = threadIdx.x; j < nvec; j += 256) dst[j] = encode8(__ldg(src + j), rs.r);
+  for (int j = threadIdx.x; j < nvec; j += 256) dst[j] = encode8<F>(__ldg(src + j), rs.r);
   if (threadIdx.x == 0) S[row] = rs.s;
+}
+
+// ------------------------------------------------------------ per-tensor (E4M3)
+// One scale for a whole matrix (the FFN weights of "FP8量化在生成式推荐系统
+// OneRec-V2中的优化实践" §2.1): the same steps with a = max over all elements.
+// Three launches on the stream after S[0] is zeroed:
+//   tensor_amax_kernel   every CTA reduces max|x| over its grid-stride share
+//                        and raises S[0] with an atomic max on the float bits
+//                        (for non-negative floats the unsigned order is the
+//                        float order);
+//   quant_tensor_kernel  every CTA reads the amax from S[0], derives r and s
+//                        (the per-row formulas) and writes its codes, and s
+//                        into S[row] for rows >= 1 (S[0] is still being read);
+//   quant_tensor_finish  S[0] = s.
+// The scale is thus replicated once per row (output channel), the form the
+// per-channel GEMM epilogue consumes.
+__global__ void __launch_bounds__(256) tensor_amax_kernel(const __half* __restrict__ X, int64_t nvec,
+                                                         unsigned int* __restrict__ amax_bits) {
+  __shared__ float red[8];
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
+  const uint4* src = reinterpret_cast<const uint4*>(X);
+  float m = 0.0f;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; j < nvec;
+       j += static_cast<int64_t>(gridDim.x) * 256)
+    m = absmax8(__ldg(src + j), m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
+    atomicMax(amax_bits, __float_as_uint(m));
+  }
+}
+
+__global__ void __launch_bounds__(256) quant_tensor_kernel(const __half* __restrict__ X, int M, int64_t nvec,
+                                                          uint8_t* __restrict__ Q, float* __restrict__ S) {
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
+  const RowScale rs = row_scale_from_amax<kFmtE4M3>(S[0]);
+  const uint4* src = reinterpret_cast<const uint4*>(X);
+  uint2* dst = reinterpret_cast<uint2*>(Q);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  for (int64_t j = first; j < nvec; j += stride) dst[j] = encode8<kFmtE4M3>(__ldg(src + j), rs.r);
+  for (int64_t r = first + 1; r < M; r += stride) S[r] = rs.s;
+}
+
+__global__ void quant_tensor_finish_kernel(float* __restrict__ S) {
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
+  if (threadIdx.x == 0 && blockIdx.x == 0) S[0] = row_scale_from_amax<kFmtE4M3>(S[0]).s;
 }
 
 // Diagnostic elementwise cast (same device cast as the quantizers).
@@ -167,17 +232,18 @@ inline cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cu
 }
 
 // Host-side launcher: picks (TPR, VPT) so one row fits in registers.
+template <int F = kFmtE4M3>
 inline cudaError_t launch_quant_rows(const __half* X, int M, int K, uint8_t* Q, float* S, cudaStream_t st) {
   const int nvec = K / 8;
   int tpr = 32;
   while (tpr < 256 && tpr * 8 < nvec) tpr *= 2;
   const int vpt_needed = (nvec + tpr - 1) / tpr;
-  if (vpt_needed > 8) return launch_pdl(quant_rows_long_kernel, dim3(M), dim3(256), st, X, M, K, Q, S);
+  if (vpt_needed > 8) return launch_pdl(quant_rows_long_kernel<F>, dim3(M), dim3(256), st, X, M, K, Q, S);
   const int rows_per_cta = 256 / tpr;
   const dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
   const int vpt = vpt_needed <= 1 ? 1 : vpt_needed <= 2 ? 2 : vpt_needed <= 4 ? 4 : 8;
 #define FP8Q_QR_CASE(T, V) \
-  if (tpr == T && vpt == V) return launch_pdl(quant_rows_kernel<T, V>, grid, dim3(256), st, X, M, K, Q, S);
+  if (tpr == T && vpt == V) return launch_pdl(quant_rows_kernel<T, V, F>, grid, dim3(256), st, X, M, K, Q, S);
   FP8Q_QR_CASE(32, 1) FP8Q_QR_CASE(32, 2) FP8Q_QR_CASE(32, 4) FP8Q_QR_CASE(32, 8)
   FP8Q_QR_CASE(64, 8) FP8Q_QR_CASE(128, 8) FP8Q_QR_CASE(256, 8)
 #undef FP8Q_QR_CASE

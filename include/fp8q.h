@@ -173,6 +173,58 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x,
                                     int64_t N, int64_t K,
                                     void* Y_f16, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Variants described on the pages [P2]: E5M2 activations (§2.2) and a
+ * per-tensor weight scale for the FFN linears (§2.1).  Same conventions as
+ * above.
+ */
+
+/* FP8 code format of the activations: E4M3 (the path's format) or E5M2
+ * [P2 §2.2: 5 exponent and 2 mantissa bits; largest finite value 57344]. */
+typedef enum {
+  FP8Q_FMT_E4M3 = 0,
+  FP8Q_FMT_E5M2 = 1
+} fp8q_format;
+
+/*
+ * fp8q_quantize_rows_dynamic with the code format chosen by fmt.  For
+ * FP8Q_FMT_E5M2 the steps use max_code = 57344 instead of 448:
+ * r = 57344 / a', s = a' / 57344, q = E5M2(fl32(x * r)), round-to-nearest-
+ * even, saturating to ±57344 (never infinity).  Any other fmt value returns
+ * FP8Q_ERR_INVALID_ARG.
+ */
+fp8q_status fp8q_quantize_rows_dynamic_fmt(const void* X_f16, int64_t M, int64_t K, fp8q_format fmt,
+                                           uint8_t* Xq, float* s_x, void* stream);
+
+/*
+ * Per-tensor weight quantization  [P2 §2.1: the FFN linear transforms use
+ * per-tensor quantization].  W_f16 [N,K] fp16 in; Wq [N,K] uint8 E4M3 and
+ * s_w [N] fp32 out.  One scale for the whole matrix: a' = max(max |W|,
+ * 1e-12), then r, s and the codes as for fp8q_quantize_rows_dynamic; the
+ * scale is written to every s_w[n], so the result feeds fp8q_linear as is.
+ * N > 0.  s_w[0] serves as the reduction word while the call runs (it is
+ * zeroed with cudaMemsetAsync on `stream`, then three kernels follow).
+ */
+fp8q_status fp8q_quantize_weight_per_tensor(const void* W_f16, int64_t N, int64_t K,
+                                            uint8_t* Wq, float* s_w, void* stream);
+
+/*
+ * fp8q_linear with the activation codes Xq in format x_fmt (weights E4M3):
+ * the tensor cores multiply E5M2 x E4M3 directly (tcgen05 kind::f8f6f4
+ * takes the two operand formats separately); everything else is identical.
+ */
+fp8q_status fp8q_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, const float* s_x,
+                            const uint8_t* Wq, const float* s_w,
+                            int64_t M, int64_t N, int64_t K,
+                            void* Y_f16, void* stream);
+
+/* fp8q_moe_grouped_linear with the activation codes Xq in format x_fmt. */
+fp8q_status fp8q_moe_grouped_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, const float* s_x,
+                                        const int32_t* offsets, int32_t E, int64_t rows,
+                                        const uint8_t* Wq, const float* s_w,
+                                        int64_t N, int64_t K,
+                                        void* Y_f16, void* stream);
+
 /*
  * Diagnostic: the device E4M3 cast on its own, out[i] = E4M3(x[i]) with the
  * same rounding as the quantizers (RNE, saturating to ±448).  n >= 0,

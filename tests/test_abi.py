@@ -118,3 +118,27 @@ def test_quantized_linear_rejects(L, M, N, K, ws):
 
 def test_quantized_linear_zero_rows_noop(L):
     assert _lib.fp8q_quantized_linear(0, 0, 0, 0, 16, 32, 0, 0, 0, 0) == _lib.FP8Q_OK
+
+
+def test_format_variants_reject_bad_format_and_shapes(L):
+    a = 0x1000
+    # unknown format codes are refused before anything runs
+    assert _lib.fp8q_quantize_rows_dynamic_fmt(a, 4, 32, 2, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_quantize_rows_dynamic_fmt(a, 4, 32, -1, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_linear_fmt(a, 2, a, a, a, 4, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_moe_grouped_linear_fmt(a, 7, a, a, 4, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    # valid format, bad shapes or pointers
+    assert _lib.fp8q_quantize_rows_dynamic_fmt(a, 4, 24, _lib.FP8Q_FMT_E5M2, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_quantize_rows_dynamic_fmt(a, 0, 32, _lib.FP8Q_FMT_E5M2, 0, 0, 0) == _lib.FP8Q_OK
+    assert _lib.fp8q_linear_fmt(a, _lib.FP8Q_FMT_E5M2, a, BAD, a, 4, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_linear_fmt(0, _lib.FP8Q_FMT_E5M2, 0, 0, 0, 0, 16, 32, 0, 0) == _lib.FP8Q_OK
+    assert _lib.fp8q_moe_grouped_linear_fmt(a, _lib.FP8Q_FMT_E5M2, a, a, 0, 8, a, a, 16, 32, a, 0) \
+        == _lib.FP8Q_ERR_INVALID_ARG
+
+
+def test_per_tensor_rejects(L):
+    a = 0x1000
+    assert _lib.fp8q_quantize_weight_per_tensor(a, 0, 32, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_quantize_weight_per_tensor(a, 4, 40, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_quantize_weight_per_tensor(BAD, 4, 32, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_quantize_weight_per_tensor(a, 4, 32, a, 0, 0) == _lib.FP8Q_ERR_INVALID_ARG

@@ -18,16 +18,18 @@ Sources (two web pages describing the same method):
 Where the pages leave a step open the reading taken is stated beside the code
 (rounding: round-to-nearest-even, saturating to ±448; eps = 1e-12; scale
 stored as amax/448 and codes produced with one fp32 multiply by 448/amax).
-Variants from [P2]: E5M2 activations (§2.2; max 57344, same steps) and
-per-tensor weight scales for the FFN linears (§2.1).
+Variants from [P2]: E5M2 activations (§2.2; max 57344, same steps),
+per-tensor weight scales for the FFN linears (§2.1) and 128x128 block-wise
+weight scales for the MoE experts (§2.1, §2.2).
 
 Every function here is pinned by tests against closed forms, hand-worked
 rows, a library cast routine and brute force; none is "parity unpinned".
 """
 from .e4m3 import E4M3_MAX, e4m3_decode, e4m3_encode
 from .e5m2 import E5M2_MAX, e5m2_decode, e5m2_encode
-from .quant import EPS, quant_rows, quant_tensor
-from .linear import linear_ref, moe_ref, linear_f64_unquantized
+from .quant import EPS, quant_blocks, quant_rows, quant_tensor
+from .linear import linear_blockscaled_ref, linear_f64_unquantized, linear_ref, moe_blockscaled_ref, moe_ref
 
 __all__ = ["E4M3_MAX", "e4m3_decode", "e4m3_encode", "E5M2_MAX", "e5m2_decode", "e5m2_encode",
-           "EPS", "quant_rows", "quant_tensor", "linear_ref", "moe_ref", "linear_f64_unquantized"]
+           "EPS", "quant_rows", "quant_tensor", "quant_blocks", "linear_ref", "moe_ref",
+           "linear_blockscaled_ref", "moe_blockscaled_ref", "linear_f64_unquantized"]

@@ -13,6 +13,12 @@ any FP32 accumulation order:
 With activations in E5M2 (['FP8量化在生成式推荐系统OneRec-V2中的优化实践'
 §2.2]) only dec(Xq) changes: x_fmt names the activation codec.
 
+Block-scaled weights (same page, §2.1, MoE: 128x128 blocks): each K block j
+of 128 inputs contributes its partial product times the scale of the weight
+block (n // 128, j):
+    Y[m,n] = fp16_rne( s_x[m] * sum_j s_w[n // 128, j] * sum_{k in block j} dec(Xq[m,k]) * dec(Wq[n,k]) )
+(float64 throughout).
+
 No bias term (the pages name none).  The float64 -> float16 cast is NumPy's
 direct, correctly rounded conversion (round half to even, overflow to inf).
 
@@ -61,3 +67,33 @@ def moe_ref(Xq, s_x, offsets, Wq, s_w, x_fmt: str = "e4m3") -> np.ndarray:
 def linear_f64_unquantized(X, W) -> np.ndarray:
     """X @ W^T in float64 on the original (unquantized) values, for error-bound pins."""
     return np.asarray(X, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T
+
+
+def linear_blockscaled_ref(Xq, s_x, Wq, s_wb, block: int = 128) -> np.ndarray:
+    """Xq uint8 [M,K], s_x f32 [M], Wq uint8 [N,K], s_wb f32 [ceil(N/b), ceil(K/b)] -> float16 [M,N]."""
+    Dx = e4m3_decode(Xq)
+    Dw = e4m3_decode(Wq)
+    M, K = Dx.shape
+    N = Dw.shape[0]
+    s_wb = np.asarray(s_wb, dtype=np.float64)
+    acc = np.zeros((M, N))
+    for j in range(-(-K // block)):
+        part = Dx[:, j * block:(j + 1) * block] @ Dw[:, j * block:(j + 1) * block].T   # [M, N]
+        col_scale = s_wb[np.arange(N) // block, j]                                        # [N]
+        acc += part * col_scale[None, :]
+    return (acc * np.asarray(s_x, dtype=np.float64)[:, None]).astype(np.float16)
+
+
+def moe_blockscaled_ref(Xq, s_x, offsets, Wq, s_wb, block: int = 128) -> np.ndarray:
+    """Grouped linear with block-scaled expert weights: Wq uint8 [E,N,K], s_wb f32 [E, ceil(N/b), ceil(K/b)]."""
+    offsets = np.asarray(offsets, dtype=np.int64)
+    E, N, _ = np.asarray(Wq).shape
+    R = np.asarray(Xq).shape[0]
+    if offsets.shape != (E + 1,) or offsets[0] != 0 or offsets[-1] != R or np.any(np.diff(offsets) < 0):
+        raise ValueError("offsets must be non-decreasing, start at 0 and end at the row count")
+    Y = np.zeros((R, N), dtype=np.float16)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            Y[lo:hi] = linear_blockscaled_ref(Xq[lo:hi], s_x[lo:hi], Wq[e], s_wb[e], block)
+    return Y

@@ -24,6 +24,12 @@ quantization; §2.2 keeps the activations per token, so the per-tensor scale
 is the weight's]: a is the maximum over the whole matrix, then the same r, s
 and codes; the one scale is returned replicated once per row (output
 channel), the form the per-channel linear consumes.
+
+Block-wise variant [same page, §2.1: the MoE expert grouped GEMM is
+quantized "block-wise 128x128"; §2.2: block-aligned quantization for MoE]:
+the weight matrix is cut into blocks of 128 output channels x 128 input
+elements (ragged at the edges); each block gets its own a, r, s and codes
+by the same steps; activations stay per token.
 """
 from __future__ import annotations
 
@@ -71,3 +77,25 @@ def quant_tensor(A) -> tuple[np.ndarray, np.ndarray]:
         raise ValueError("quant_tensor expects a 2-D matrix")
     a = np.float32(np.max(np.abs(a32))) if a32.size else np.float32(0.0)
     return _quant_with_amax(a32, np.full(a32.shape[0], a, dtype=np.float32), "e4m3")
+
+
+def quant_blocks(A, block: int = 128) -> tuple[np.ndarray, np.ndarray]:
+    """Block-wise E4M3: A [R, K] -> (codes uint8 [R, K], scales float32 [ceil(R/b), ceil(K/b)]).
+
+    Block (i, j) covers rows i*b .. i*b+b-1 and columns j*b .. j*b+b-1.
+    """
+    a32 = np.asarray(A).astype(np.float32)
+    if a32.ndim != 2:
+        raise ValueError("quant_blocks expects a 2-D matrix")
+    R, K = a32.shape
+    nb_r, nb_k = -(-R // block), -(-K // block)
+    codes = np.zeros((R, K), dtype=np.uint8)
+    scales = np.zeros((nb_r, nb_k), dtype=np.float32)
+    for i in range(nb_r):
+        for j in range(nb_k):
+            blk = a32[i * block:(i + 1) * block, j * block:(j + 1) * block]
+            a = np.float32(np.max(np.abs(blk))) if blk.size else np.float32(0.0)
+            c, s = _quant_with_amax(blk, np.full(blk.shape[0], a, dtype=np.float32), "e4m3")
+            codes[i * block:(i + 1) * block, j * block:(j + 1) * block] = c
+            scales[i, j] = s[0] if s.size else np.float32(np.maximum(a, EPS) / np.float32(E4M3_MAX))
+    return codes, scales

@@ -147,7 +147,11 @@ class Plan:
         self.device = device
         # activation codes E4M3 (the path) or E5M2 (variant); weight scales per channel or per tensor (variant)
         self.x_fmt = x_fmt
-        self.weights = weights if kind == "dense" else "channel"   # per-tensor scales: the dense (FFN) variant
+        # per-tensor scales: the dense (FFN) variant; 128x128 block scales: the MoE variant
+        if (weights == "tensor" and kind != "dense") or (weights == "block" and kind == "dense"):
+            raise SystemExit(f"--weight-scales {weights} applies to "
+                             f"{'dense' if weights == 'tensor' else 'moe'} workloads only")
+        self.weights = weights
         self.fmt = _lib.FORMATS[x_fmt]
         # Up to 16 token rows the library quantizes inside the GEMM (one launch; E4M3 only).
         self.fused = fused and kind == "dense" and x_fmt == "e4m3" and tensors[0].shape[0] <= fq.FUSED_MAX_ROWS
@@ -178,8 +182,9 @@ class Plan:
             else:
                 b["X"] = Xp.to(device)
                 b["off"] = torch.from_numpy(offsets).to(device)
-                b["Wuq"], b["swu"] = fq.quantize_weight_per_channel(Wu.to(device))
-                b["Wdq"], b["swd"] = fq.quantize_weight_per_channel(Wd.to(device))
+                qw = fq.quantize_weight_blockwise if weights == "block" else fq.quantize_weight_per_channel
+                b["Wuq"], b["swu"] = qw(Wu.to(device))
+                b["Wdq"], b["swd"] = qw(Wd.to(device))
                 b["Xq"] = torch.empty((self.R, self.D), dtype=torch.uint8, device=device)
                 b["sx"] = torch.empty((self.R,), dtype=torch.float32, device=device)
                 b["H"] = torch.empty((self.R, self.F), dtype=torch.float16, device=device)
@@ -211,10 +216,14 @@ class Plan:
             return [(M * K * 3 + 4 * M, 0.0),
                     (M * K + N * K + 4 * M + 4 * N + 2 * M * N, 2.0 * M * N * K)]
         R, D, F, E = self.R, self.D, self.F, self.E
+        if self.weights == "block":   # one scale per 128 x 128 weight block
+            su, sd = 4 * E * (-(-F // 128)) * (-(-D // 128)), 4 * E * (-(-D // 128)) * (-(-F // 128))
+        else:
+            su, sd = 4 * E * F, 4 * E * D
         return [(R * D * 3 + 4 * R, 0.0),
-                (R * D + E * F * D + 4 * R + 4 * E * F + 2 * R * F, 2.0 * R * F * D),
+                (R * D + E * F * D + 4 * R + su + 2 * R * F, 2.0 * R * F * D),
                 (R * F * 3 + 4 * R, 0.0),
-                (R * F + E * D * F + 4 * R + 4 * E * D + 2 * R * D, 2.0 * R * D * F)]
+                (R * F + E * D * F + 4 * R + sd + 2 * R * D, 2.0 * R * D * F)]
 
     def launch(self, i, k):
         """Launch kernel k of step i (raw C ABI, integer pointers)."""
@@ -232,10 +241,17 @@ class Plan:
             if k == 0:
                 s = L.fp8q_quantize_rows_dynamic_fmt(p["X"], self.R, self.D, self.fmt, p["Xq"], p["sx"], st)
             elif k == 1:
-                s = L.fp8q_moe_grouped_linear_fmt(p["Xq"], self.fmt, p["sx"], p["off"], self.E, self.R, p["Wuq"],
-                                                  p["swu"], self.F, self.D, p["H"], st)
+                if self.weights == "block":
+                    s = L.fp8q_moe_grouped_linear_blockscaled(p["Xq"], p["sx"], p["off"], self.E, self.R, p["Wuq"],
+                                                              p["swu"], self.F, self.D, p["H"], st)
+                else:
+                    s = L.fp8q_moe_grouped_linear_fmt(p["Xq"], self.fmt, p["sx"], p["off"], self.E, self.R,
+                                                      p["Wuq"], p["swu"], self.F, self.D, p["H"], st)
             elif k == 2:
                 s = L.fp8q_quantize_rows_dynamic_fmt(p["H"], self.R, self.F, self.fmt, p["Hq"], p["sh"], st)
+            elif self.weights == "block":
+                s = L.fp8q_moe_grouped_linear_blockscaled(p["Hq"], p["sh"], p["off"], self.E, self.R, p["Wdq"],
+                                                          p["swd"], self.D, self.F, p["Y"], st)
             else:
                 s = L.fp8q_moe_grouped_linear_fmt(p["Hq"], self.fmt, p["sh"], p["off"], self.E, self.R, p["Wdq"],
                                                   p["swd"], self.D, self.F, p["Y"], st)
@@ -360,7 +376,7 @@ def timed_e2e(plan, tensors, steps):
 # --------------------------------------------------------------------------- oracle arm
 def oracle_sampler(kind, tensors, m_rows, n_rows, x_fmt="e4m3", weights="channel"):
     """A callable running the oracle on an (m_rows x n_rows) output sample; returns its FLOPs."""
-    from oracle import linear_ref, quant_rows, quant_tensor
+    from oracle import linear_blockscaled_ref, linear_ref, quant_blocks, quant_rows, quant_tensor
     if kind == "dense":
         X, W = tensors
         Xn = X.numpy()
@@ -385,9 +401,21 @@ def oracle_sampler(kind, tensors, m_rows, n_rows, x_fmt="e4m3", weights="channel
     lo = int(offsets[e])
     cnt = min(m_rows, int(offsets[e + 1]) - lo)
     Xn = Xp.numpy()[lo:lo + cnt]
+    D = Xn.shape[1]
+    if weights == "block":
+        Wuq, swu = quant_blocks(Wu[e].numpy()[:n_rows])
+        Wdq, swd = quant_blocks(Wd[e].numpy()[:n_rows, :n_rows])
+
+        def run():
+            xq, sx = quant_rows(Xn)
+            h = linear_blockscaled_ref(xq, sx, Wuq, swu)
+            hq, sh = quant_rows(h)
+            linear_blockscaled_ref(hq, sh, Wdq, swd)
+            return 2.0 * cnt * Wuq.shape[0] * D + 2.0 * cnt * n_rows * hq.shape[1]
+        return run, (f"expert {e}: {cnt} rows through up ({n_rows} channels) and down ({n_rows} channels), "
+                     "128x128 block-scaled weights")
     Wuq, swu = quant_rows(Wu[e].numpy()[:n_rows])
     Wdq, swd = quant_rows(Wd[e].numpy()[:, :])
-    D = Xn.shape[1]
 
     def run():
         xq, sx = quant_rows(Xn, x_fmt)
@@ -480,7 +508,7 @@ def run_reference(args, world, rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": desc, "sample_per_step": sample, "parallelism": "host cores (rank 0 only)",
                        "activation_format": args.x_fmt,
-                       "weight_scales": "per-" + (args.weight_scales if kind == "dense" else "channel")},
+                       "weight_scales": "per-" + args.weight_scales},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -619,8 +647,9 @@ def main(argv=None):
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of a CUDA graph")
     ap.add_argument("--x-fmt", default="e4m3", choices=["e4m3", "e5m2"],
                     help="activation code format (e5m2: the pages' activation-format variant)")
-    ap.add_argument("--weight-scales", default="channel", choices=["channel", "tensor"],
-                    help="weight scale granularity for dense workloads (tensor: the pages' FFN variant)")
+    ap.add_argument("--weight-scales", default="channel", choices=["channel", "tensor", "block"],
+                    help="weight scale granularity: channel (the path), tensor (the pages' FFN variant, dense "
+                         "workloads) or block (128x128, the pages' MoE variant, moe workload)")
     ap.add_argument("--fused", action="store_true",
                     help="one fused quantize+linear launch per step where it applies (<= 16 rows); "
                          "default: the two launches, measured faster on B200")

@@ -13,8 +13,9 @@ missing library raises ImportError at the first call.
     Y = moe_grouped_linear(Xq, s_x, offsets, Wq_e, s_w_e)
 
 Variants from the pages: activations in E5M2 (quantize_rows_dynamic(X,
-fmt="e5m2") with linear(..., x_fmt="e5m2")) and per-tensor weight scales
-(quantize_weight_per_tensor).
+fmt="e5m2") with linear(..., x_fmt="e5m2")), per-tensor weight scales
+(quantize_weight_per_tensor) and 128x128 block-scaled MoE expert weights
+(quantize_weight_blockwise with moe_grouped_linear_blockscaled).
 """
 from __future__ import annotations
 
@@ -25,7 +26,8 @@ from ._lib import Fp8qError, check, lib
 
 __all__ = [
     "Fp8qError", "lib", "quantize_rows_dynamic", "quantize_weight_per_channel", "quantize_weight_per_tensor",
-    "linear", "moe_grouped_linear", "quantized_linear", "e4m3_encode_f32", "device_error", "set_gemm_tuning",
+    "quantize_weight_blockwise", "linear", "moe_grouped_linear", "moe_grouped_linear_blockscaled",
+    "quantized_linear", "e4m3_encode_f32", "device_error", "set_gemm_tuning",
 ]
 
 
@@ -168,6 +170,46 @@ def moe_grouped_linear(Xq: torch.Tensor, s_x: torch.Tensor, offsets: torch.Tenso
         check(_lib.fp8q_moe_grouped_linear_fmt(Xq.data_ptr(), _fmt(x_fmt), s_x.data_ptr(), offsets.data_ptr(), E, rows,
                                                Wq.data_ptr(), s_w.data_ptr(), N, K, Y.data_ptr(), _stream(Xq)),
               "fp8q_moe_grouped_linear_fmt")
+    return Y
+
+
+BLOCK = 128
+
+
+def quantize_weight_blockwise(W: torch.Tensor):
+    """Offline 128x128 block-wise E4M3 quantization: fp16 [N,K] or [E,N,K] ->
+    (uint8 same shape, fp32 scales [..., ceil(N/128), ceil(K/128)])."""
+    _need(W, torch.float16, "W")
+    if W.dim() not in (2, 3):
+        raise ValueError("W must be [N,K] or [E,N,K]")
+    E = W.shape[0] if W.dim() == 3 else 1
+    N, K = W.shape[-2], W.shape[-1]
+    Wq = torch.empty(W.shape, dtype=torch.uint8, device=W.device)
+    s = torch.empty(W.shape[:-2] + (-(-N // BLOCK), -(-K // BLOCK)), dtype=torch.float32, device=W.device)
+    check(_lib.fp8q_quantize_weight_blockwise(W.data_ptr(), E, N, K, Wq.data_ptr(), s.data_ptr(), _stream(W)),
+          "fp8q_quantize_weight_blockwise")
+    return Wq, s
+
+
+def moe_grouped_linear_blockscaled(Xq: torch.Tensor, s_x: torch.Tensor, offsets: torch.Tensor, Wq: torch.Tensor,
+                                   s_wb: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Expert-grouped FP8 linear with 128x128 block-scaled expert weights
+    (Wq [E,N,K] and s_wb [E, ceil(N/128), ceil(K/128)] from
+    quantize_weight_blockwise); per-token activation scales."""
+    _need(Xq, torch.uint8, "Xq", 2)
+    _need(s_x, torch.float32, "s_x", 1)
+    _need(offsets, torch.int32, "offsets", 1)
+    _need(Wq, torch.uint8, "Wq", 3)
+    _need(s_wb, torch.float32, "s_wb", 3)
+    rows, K = Xq.shape
+    E, N, K2 = Wq.shape
+    if (K2 != K or offsets.shape[0] != E + 1 or s_x.shape[0] != rows
+            or tuple(s_wb.shape) != (E, -(-N // BLOCK), -(-K // BLOCK))):
+        raise ValueError("shape mismatch")
+    Y = out if out is not None else torch.empty((rows, N), dtype=torch.float16, device=Xq.device)
+    check(_lib.fp8q_moe_grouped_linear_blockscaled(Xq.data_ptr(), s_x.data_ptr(), offsets.data_ptr(), E, rows,
+                                                   Wq.data_ptr(), s_wb.data_ptr(), N, K, Y.data_ptr(), _stream(Xq)),
+          "fp8q_moe_grouped_linear_blockscaled")
     return Y
 
 

@@ -57,6 +57,8 @@ SIGNATURES = {
     "fp8q_quantize_weight_per_tensor": (_INT, [_P, _I64, _I64, _P, _P, _P]),
     "fp8q_linear_fmt": (_INT, [_P, _INT, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "fp8q_moe_grouped_linear_fmt": (_INT, [_P, _INT, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
+    "fp8q_quantize_weight_blockwise": (_INT, [_P, _I32, _I64, _I64, _P, _P, _P]),
+    "fp8q_moe_grouped_linear_blockscaled": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_e4m3_encode_f32": (_INT, [_P, _I64, _P, _P]),
     "fp8q_set_gemm_tuning": (_INT, [_INT, _INT, _INT]),
     "fp8q_selftest_wait_timeout": (_INT, [ctypes.c_uint32, _P]),
@@ -138,6 +140,14 @@ def fp8q_linear_fmt(Xq, x_fmt, s_x, Wq, s_w, M, N, K, Y, stream):
 
 def fp8q_moe_grouped_linear_fmt(Xq, x_fmt, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream):
     return lib().fp8q_moe_grouped_linear_fmt(Xq, x_fmt, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream)
+
+
+def fp8q_quantize_weight_blockwise(W, E, N, K, Wq, s_wb, stream):
+    return lib().fp8q_quantize_weight_blockwise(W, E, N, K, Wq, s_wb, stream)
+
+
+def fp8q_moe_grouped_linear_blockscaled(Xq, s_x, offsets, E, rows, Wq, s_wb, N, K, Y, stream):
+    return lib().fp8q_moe_grouped_linear_blockscaled(Xq, s_x, offsets, E, rows, Wq, s_wb, N, K, Y, stream)
 
 
 def fp8q_e4m3_encode_f32(x, n, out, stream):

@@ -16,6 +16,7 @@
 #include "gemm_fp8.cuh"
 #include "gemm_fp8_pair.cuh"
 #include "gemm_fp8_splitk.cuh"
+#include "gemm_fp8_blockscaled.cuh"
 #include "quant_rows.cuh"
 
 namespace fp8q {
@@ -795,6 +796,76 @@ fp8q_status fp8q_moe_grouped_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, co
   }
   const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBNGrouped - 1) / kBNGrouped);
   return launch_gemm<true>(Xq, rows, Wq, int64_t(E) * N, p, tiles, static_cast<cudaStream_t>(stream));
+}
+
+fp8q_status fp8q_quantize_weight_blockwise(const void* W_f16, int32_t E, int64_t N, int64_t K, uint8_t* Wq,
+                                           float* s_wb, void* stream) {
+  if (E < 1 || E > kMaxExperts) return invalid("E must be in [1, 1024]");
+  if (N <= 0 || N > kMaxDim || int64_t(E) * N > kMaxDim) return invalid("N must be positive, E*N < 2^31");
+  fp8q_status s = check_quant_args(W_f16, int64_t(E) * N, K, Wq, s_wb);
+  if (s != FP8Q_OK) return s;
+  const int NB = static_cast<int>((N + kBsBlk - 1) / kBsBlk);
+  const int KB = static_cast<int>((K + kBsBlk - 1) / kBsBlk);
+  if (KB > 65535) return invalid("K too large for the block grid");
+  const cudaError_t e = launch_pdl(quant_blocks_kernel, dim3(E * NB, KB), dim3(256), static_cast<cudaStream_t>(stream),
+                                   static_cast<const __half*>(W_f16), static_cast<int>(N), static_cast<int>(K), NB, KB,
+                                   Wq, s_wb);
+  if (e != cudaSuccess) return cuda_fail(e, "quant_blocks launch");
+  return FP8Q_OK;
+}
+
+fp8q_status fp8q_moe_grouped_linear_blockscaled(const uint8_t* Xq, const float* s_x, const int32_t* offsets,
+                                                int32_t E, int64_t rows, const uint8_t* Wq, const float* s_wb,
+                                                int64_t N, int64_t K, void* Y_f16, void* stream) {
+  if (E < 1 || E > kBsMaxExperts) return invalid("E must be in [1, 128] for block-scaled weights");
+  if (rows < 0 || rows > kMaxDim) return invalid("rows out of range");
+  if (N <= 0 || N % 8 != 0 || int64_t(E) * N > kMaxDim) return invalid("N must be positive, a multiple of 8, E*N < 2^31");
+  if (K <= 0 || K > kMaxDim || K % 16 != 0) return invalid("K must be positive and a multiple of 16");
+  if (offsets == nullptr || (reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return invalid("offsets pointer");
+  if (rows == 0) return FP8Q_OK;
+  if (!aligned16(Xq) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_wb) || !aligned16(Y_f16))
+    return invalid("null or non-16-byte-aligned pointer");
+  int dev = 0, sms = 0;
+  cudaError_t e = current_device_info(&dev, &sms);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  GemmParams p = {};
+  p.s_x = s_x;
+  p.s_w = s_wb;   // block scales [E, ceil(N/128), ceil(K/128)]
+  p.Y = static_cast<__half*>(Y_f16);
+  p.offsets = offsets;
+  p.rows = static_cast<int>(rows);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.E = E;
+  p.tail_q = 1;
+  p.x_fmt = FP8Q_FMT_E4M3;
+  constexpr int kStagesBs = 4;
+  using L = BsLayout<kStagesBs>;
+  CUtensorMap ta, tb, ty;
+  fp8q_status s = make_operand_map(&ta, Xq, rows, K, kBM);
+  if (s != FP8Q_OK) return s;
+  s = make_operand_map(&tb, Wq, int64_t(E) * N, K, kBsBN);
+  if (s != FP8Q_OK) return s;
+  s = make_output_map(&ty, p.Y, rows, N);
+  if (s != FP8Q_OK) return s;
+  e = ensure_smem<fp8_gemm_blockscaled_kernel<kStagesBs>>(L::smem_bytes(kBsMaxExperts), dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(blockscaled)");
+  const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBsBN - 1) / kBsBN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  e = launch_ex(fp8_gemm_blockscaled_kernel<kStagesBs>, dim3(grid), dim3(kBsThreads), L::smem_bytes(E),
+                static_cast<cudaStream_t>(stream), 1, true, ta, tb, ty, p);
+  if (e != cudaSuccess) {
+    cudaFuncAttributes fa = {};
+    (void)cudaFuncGetAttributes(&fa, fp8_gemm_blockscaled_kernel<kStagesBs>);
+    char msg[256];
+    std::snprintf(msg, sizeof(msg),
+                  "fp8_gemm_blockscaled_kernel launch (%d threads, %zu B dynamic smem; kernel: %d regs, max %d "
+                  "threads, %zu B static smem, max dynamic %d)",
+                  kBsThreads, L::smem_bytes(E), fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes,
+                  fa.maxDynamicSharedSizeBytes);
+    return cuda_fail(e, msg);
+  }
+  return FP8Q_OK;
 }
 
 fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* stream) {

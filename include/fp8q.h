@@ -174,9 +174,10 @@ fp8q_status fp8q_moe_grouped_linear(const uint8_t* Xq, const float* s_x,
                                     void* Y_f16, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Variants described on the pages [P2]: E5M2 activations (§2.2) and a
- * per-tensor weight scale for the FFN linears (§2.1).  Same conventions as
- * above.
+ * Variants described on the pages [P2]: E5M2 activations (§2.2), a
+ * per-tensor weight scale for the FFN linears (§2.1) and 128 x 128
+ * block-wise weight scales for the MoE experts (§2.1, §2.2).  Same
+ * conventions as above.
  */
 
 /* FP8 code format of the activations: E4M3 (the path's format) or E5M2
@@ -217,6 +218,32 @@ fp8q_status fp8q_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, const float* s
                             const uint8_t* Wq, const float* s_w,
                             int64_t M, int64_t N, int64_t K,
                             void* Y_f16, void* stream);
+
+/*
+ * Block-wise weight quantization  [P2 §2.1: the MoE expert grouped GEMM is
+ * quantized "block-wise 128x128"; §2.2: block-aligned MoE quantization].
+ * W_f16 [E,N,K] fp16 (E = 1 for one matrix) in; Wq [E,N,K] uint8 E4M3 and
+ * s_wb [E, ceil(N/128), ceil(K/128)] fp32 out.  Each 128 x 128 block of an
+ * expert's [N,K] weights (ragged at the edges; blocks never span experts)
+ * gets its own a', r, s and codes by the per-row rule.  1 <= E <= 1024.
+ */
+fp8q_status fp8q_quantize_weight_blockwise(const void* W_f16, int32_t E, int64_t N, int64_t K,
+                                           uint8_t* Wq, float* s_wb, void* stream);
+
+/*
+ * MoE expert grouped FP8 linear with block-scaled expert weights (from
+ * fp8q_quantize_weight_blockwise) and per-token activation scales:
+ *   Y[r,n] = fp16( s_x[r] * sum_j s_wb[e, n/128, j] * P_j[r,n] ),
+ *   P_j = FP32 tensor-core sum over the 128 inputs of K block j,
+ * e the expert of row r (offsets as for fp8q_moe_grouped_linear).  Each K
+ * block's partial is scaled and accumulated in FP32 registers (the sum over
+ * j runs in K-block order).  1 <= E <= 128.
+ */
+fp8q_status fp8q_moe_grouped_linear_blockscaled(const uint8_t* Xq, const float* s_x,
+                                                const int32_t* offsets, int32_t E, int64_t rows,
+                                                const uint8_t* Wq, const float* s_wb,
+                                                int64_t N, int64_t K,
+                                                void* Y_f16, void* stream);
 
 /* fp8q_moe_grouped_linear with the activation codes Xq in format x_fmt. */
 fp8q_status fp8q_moe_grouped_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, const float* s_x,

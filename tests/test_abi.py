@@ -142,3 +142,19 @@ def test_per_tensor_rejects(L):
     assert _lib.fp8q_quantize_weight_per_tensor(a, 4, 40, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
     assert _lib.fp8q_quantize_weight_per_tensor(BAD, 4, 32, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
     assert _lib.fp8q_quantize_weight_per_tensor(a, 4, 32, a, 0, 0) == _lib.FP8Q_ERR_INVALID_ARG
+
+
+def test_blockscaled_rejects(L):
+    a = 0x1000
+    assert _lib.fp8q_quantize_weight_blockwise(a, 0, 16, 32, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_quantize_weight_blockwise(a, 2, 0, 32, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_quantize_weight_blockwise(a, 2, 16, 40, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert _lib.fp8q_quantize_weight_blockwise(BAD, 2, 16, 32, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    mo = _lib.fp8q_moe_grouped_linear_blockscaled
+    assert mo(a, a, a, 129, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG      # E > 128
+    assert mo(a, a, a, 0, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert mo(a, a, a, 4, 8, a, a, 12, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG       # N % 8
+    assert mo(a, a, a, 4, 8, a, a, 16, 24, a, 0) == _lib.FP8Q_ERR_INVALID_ARG       # K % 16
+    assert mo(a, a, 0x1002, 4, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG  # offsets alignment
+    assert mo(a, a, a, 4, 8, a, BAD, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert mo(0, 0, a, 4, 0, 0, 0, 16, 32, 0, 0) == _lib.FP8Q_OK                    # no rows

@@ -97,3 +97,20 @@ def moe_blockscaled_ref(Xq, s_x, offsets, Wq, s_wb, block: int = 128) -> np.ndar
         if hi > lo:
             Y[lo:hi] = linear_blockscaled_ref(Xq[lo:hi], s_x[lo:hi], Wq[e], s_wb[e], block)
     return Y
+
+
+def moe_gather_ref(Xq_tok, s_x_tok, row_token, offsets, Wq, s_w) -> np.ndarray:
+    """Grouped linear whose rows are gathered from the token matrix.
+
+    [P1 关键证据 item 2; P2 §3.2, inter-expert pipeline]: the routed rows of
+    the MoE layer are the tokens themselves, so the activations are quantized
+    once per token (Xq_tok uint8 [T,K], s_x_tok f32 [T]) and row r of the
+    grouped product (rows in expert order, offsets as in moe_ref) reads token
+    row_token[r].  Per-row quantization commutes with the row gather, so this
+    equals moe_ref on the gathered (permuted) rows.
+    """
+    row_token = np.asarray(row_token, dtype=np.int64)
+    Xq_tok = np.asarray(Xq_tok)
+    if row_token.size and (row_token.min() < 0 or row_token.max() >= Xq_tok.shape[0]):
+        raise ValueError("row_token out of range")
+    return moe_ref(Xq_tok[row_token], np.asarray(s_x_tok)[row_token], offsets, Wq, s_w)

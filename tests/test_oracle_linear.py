@@ -215,3 +215,40 @@ def test_per_tensor_weights_linear_error_bound():
     Y = linear_ref(Xq, sx, Wq, sw)
     err = np.abs(Y.astype(np.float64) - linear_f64_unquantized(X, W))
     assert np.all(err <= quant_error_bound(X, W, sx, sw, Y))
+
+
+# ---------------------------------------------------------------------------
+# Row gather of the MoE grouped linear (tokens quantized once, rows read by index).
+
+def test_per_row_quantization_commutes_with_row_gather():
+    rng = np.random.default_rng(61)
+    X = (rng.standard_normal((40, 96)) * np.exp(rng.uniform(-3, 3, (40, 1)))).astype(np.float16)
+    idx = rng.integers(0, 40, size=70)                 # repeats, like top-2 routing
+    q_all, s_all = quant_rows(X)
+    q_sel, s_sel = quant_rows(X[idx])
+    np.testing.assert_array_equal(q_all[idx], q_sel)
+    np.testing.assert_array_equal(s_all[idx].view(np.uint32), s_sel.view(np.uint32))
+
+
+def test_moe_gather_matches_permuted_rows_and_identity():
+    from fp8_quantized_generative_b200 import workloads as wl
+    from oracle import moe_gather_ref
+    rng = np.random.default_rng(63)
+    T, E, N, K = 24, 4, 12, 32
+    X = rng.standard_normal((T, K)).astype(np.float16)
+    logits = rng.standard_normal((T, E)).astype(np.float16)
+    experts = wl.route_top2(logits)
+    row_token, offsets = wl.group_by_expert(experts, E)
+    W = (rng.standard_normal((E, N, K)) * 0.05).astype(np.float16)
+    q = [quant_rows(W[e]) for e in range(E)]
+    Wq = np.stack([c for c, _ in q]); sw = np.stack([s for _, s in q])
+    xq, sx = quant_rows(X)
+    xq_p, sx_p = quant_rows(X[row_token])
+    got = moe_gather_ref(xq, sx, row_token, offsets, Wq, sw)
+    np.testing.assert_array_equal(got.view(np.uint16), moe_ref(xq_p, sx_p, offsets, Wq, sw).view(np.uint16))
+    # identity gather on already grouped rows
+    ident = np.arange(len(row_token))
+    np.testing.assert_array_equal(moe_gather_ref(xq_p, sx_p, ident, offsets, Wq, sw).view(np.uint16),
+                                  moe_ref(xq_p, sx_p, offsets, Wq, sw).view(np.uint16))
+    with pytest.raises(ValueError):
+        moe_gather_ref(xq, sx, np.array([0, T]), np.array([0, 2]), Wq[:1], sw[:1])

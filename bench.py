@@ -73,6 +73,12 @@ def workload_spec(name: str):
         m = wl.moe()
         return ("moe_ffn T=8192 top2 E=64 d=2048 F=1024 (16384 grouped rows)", "moe",
                 (m.X_perm, m.offsets, m.W_up, m.W_down))
+    if name == "moe_tokens":
+        # the same layer from the token matrix: tokens quantized once, the up
+        # projection gathers its rows by the router's grouping
+        m = wl.moe()
+        return ("moe_ffn T=8192 top2 E=64 d=2048 F=1024 from the 8192-token matrix (row gather)", "moe",
+                (m.X, m.offsets, m.W_up, m.W_down, np.asarray(m.token_of_row, dtype=np.int32)))
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -162,11 +168,15 @@ class Plan:
             self.flops = 2.0 * self.M * self.N * self.K
             per_set = (self.M * self.K * 3 + 4 * self.M + self.N * self.K + 4 * self.N + 2 * self.M * self.N)
         else:
-            Xp, offsets, Wu, Wd = tensors
-            self.R, self.D = Xp.shape
+            Xp, offsets, Wu, Wd = tensors[:4]
+            # gather form: Xp is the token matrix and tensors[4] the row -> token map
+            self.row_token = tensors[4] if len(tensors) > 4 else None
+            self.T = Xp.shape[0]
+            self.R = int(offsets[-1])
+            self.D = Xp.shape[1]
             self.E, self.F, _ = Wu.shape
             self.flops = 2.0 * self.R * self.F * self.D * 2
-            per_set = (self.R * self.D * 3 + 8 * self.R + 2 * self.E * self.F * self.D + 8 * self.E * self.F
+            per_set = (self.T * self.D * 3 + 8 * self.R + 2 * self.E * self.F * self.D + 8 * self.E * self.F
                        + self.R * self.F * 5 + self.R * self.D * 2)
         self.sets = max(2, math.ceil(min_rotation_bytes / per_set))
         self.bufs = []
@@ -182,11 +192,13 @@ class Plan:
             else:
                 b["X"] = Xp.to(device)
                 b["off"] = torch.from_numpy(offsets).to(device)
+                if self.row_token is not None:
+                    b["rt"] = torch.from_numpy(self.row_token).to(device)
                 qw = fq.quantize_weight_blockwise if weights == "block" else fq.quantize_weight_per_channel
                 b["Wuq"], b["swu"] = qw(Wu.to(device))
                 b["Wdq"], b["swd"] = qw(Wd.to(device))
-                b["Xq"] = torch.empty((self.R, self.D), dtype=torch.uint8, device=device)
-                b["sx"] = torch.empty((self.R,), dtype=torch.float32, device=device)
+                b["Xq"] = torch.empty((self.T, self.D), dtype=torch.uint8, device=device)
+                b["sx"] = torch.empty((self.T,), dtype=torch.float32, device=device)
                 b["H"] = torch.empty((self.R, self.F), dtype=torch.float16, device=device)
                 b["Hq"] = torch.empty((self.R, self.F), dtype=torch.uint8, device=device)
                 b["sh"] = torch.empty((self.R,), dtype=torch.float32, device=device)
@@ -204,7 +216,8 @@ class Plan:
             return ["fp8_quantized_linear_fused"]
         if self.kind == "dense":
             return ["quant_rows", "fp8_gemm"]
-        return ["quant_rows", "fp8_grouped_gemm_up", "quant_rows_h", "fp8_grouped_gemm_down"]
+        up = "fp8_grouped_gemm_up_gather" if self.row_token is not None else "fp8_grouped_gemm_up"
+        return ["quant_rows", up, "quant_rows_h", "fp8_grouped_gemm_down"]
 
     def kernel_bytes_flops(self):
         """Algorithmic bytes and FLOPs of each launch of one step."""
@@ -220,7 +233,7 @@ class Plan:
             su, sd = 4 * E * (-(-F // 128)) * (-(-D // 128)), 4 * E * (-(-D // 128)) * (-(-F // 128))
         else:
             su, sd = 4 * E * F, 4 * E * D
-        return [(R * D * 3 + 4 * R, 0.0),
+        return [(self.T * D * 3 + 4 * self.T, 0.0),
                 (R * D + E * F * D + 4 * R + su + 2 * R * F, 2.0 * R * F * D),
                 (R * F * 3 + 4 * R, 0.0),
                 (R * F + E * D * F + 4 * R + sd + 2 * R * D, 2.0 * R * D * F)]
@@ -239,7 +252,10 @@ class Plan:
                                       st)
         else:
             if k == 0:
-                s = L.fp8q_quantize_rows_dynamic_fmt(p["X"], self.R, self.D, self.fmt, p["Xq"], p["sx"], st)
+                s = L.fp8q_quantize_rows_dynamic_fmt(p["X"], self.T, self.D, self.fmt, p["Xq"], p["sx"], st)
+            elif k == 1 and self.row_token is not None:
+                s = L.fp8q_moe_grouped_linear_gather(p["Xq"], p["sx"], self.T, p["rt"], p["off"], self.E, self.R,
+                                                     p["Wuq"], p["swu"], self.F, self.D, p["H"], st)
             elif k == 1:
                 if self.weights == "block":
                     s = L.fp8q_moe_grouped_linear_blockscaled(p["Xq"], p["sx"], p["off"], self.E, self.R, p["Wuq"],
@@ -396,11 +412,12 @@ def oracle_sampler(kind, tensors, m_rows, n_rows, x_fmt="e4m3", weights="channel
             linear_ref(xq, sx, Wq[c0:c0 + n_rows], sw[c0:c0 + n_rows], x_fmt)
             return 2.0 * m_rows * n_rows * K
         return run, f"{m_rows} activation rows x {n_rows} weight rows (output block) per call"
-    Xp, offsets, Wu, Wd = tensors
+    Xp, offsets, Wu, Wd = tensors[:4]
     e = int(np.argmax(np.diff(offsets)))
     lo = int(offsets[e])
     cnt = min(m_rows, int(offsets[e + 1]) - lo)
-    Xn = Xp.numpy()[lo:lo + cnt]
+    # gather form: the expert's rows are tokens row_token[lo:lo+cnt]
+    Xn = Xp.numpy()[tensors[4][lo:lo + cnt]] if len(tensors) > 4 else Xp.numpy()[lo:lo + cnt]
     D = Xn.shape[1]
     if weights == "block":
         Wuq, swu = quant_blocks(Wu[e].numpy()[:n_rows])

@@ -26,7 +26,8 @@ from ._lib import Fp8qError, check, lib
 
 __all__ = [
     "Fp8qError", "lib", "quantize_rows_dynamic", "quantize_weight_per_channel", "quantize_weight_per_tensor",
-    "quantize_weight_blockwise", "linear", "moe_grouped_linear", "moe_grouped_linear_blockscaled",
+    "quantize_weight_blockwise", "linear", "moe_grouped_linear", "moe_grouped_linear_gather",
+    "moe_grouped_linear_blockscaled",
     "quantized_linear", "e4m3_encode_f32", "device_error", "set_gemm_tuning",
 ]
 
@@ -170,6 +171,30 @@ def moe_grouped_linear(Xq: torch.Tensor, s_x: torch.Tensor, offsets: torch.Tenso
         check(_lib.fp8q_moe_grouped_linear_fmt(Xq.data_ptr(), _fmt(x_fmt), s_x.data_ptr(), offsets.data_ptr(), E, rows,
                                                Wq.data_ptr(), s_w.data_ptr(), N, K, Y.data_ptr(), _stream(Xq)),
               "fp8q_moe_grouped_linear_fmt")
+    return Y
+
+
+def moe_grouped_linear_gather(Xq_tok: torch.Tensor, s_x_tok: torch.Tensor, row_token: torch.Tensor,
+                              offsets: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
+                              out: torch.Tensor | None = None) -> torch.Tensor:
+    """Expert-grouped FP8 linear whose row r reads token row_token[r] of the
+    per-token codes Xq_tok [T,K] (scales s_x_tok [T]); rows in expert order
+    (offsets int32 [E+1]); returns fp16 [len(row_token), N]."""
+    _need(Xq_tok, torch.uint8, "Xq_tok", 2)
+    _need(s_x_tok, torch.float32, "s_x_tok", 1)
+    _need(row_token, torch.int32, "row_token", 1)
+    _need(offsets, torch.int32, "offsets", 1)
+    _need(Wq, torch.uint8, "Wq", 3)
+    _need(s_w, torch.float32, "s_w", 2)
+    T, K = Xq_tok.shape
+    rows = row_token.shape[0]
+    E, N, K2 = Wq.shape
+    if K2 != K or offsets.shape[0] != E + 1 or tuple(s_w.shape) != (E, N) or s_x_tok.shape[0] != T:
+        raise ValueError("shape mismatch")
+    Y = out if out is not None else torch.empty((rows, N), dtype=torch.float16, device=Xq_tok.device)
+    check(_lib.fp8q_moe_grouped_linear_gather(Xq_tok.data_ptr(), s_x_tok.data_ptr(), T, row_token.data_ptr(),
+                                              offsets.data_ptr(), E, rows, Wq.data_ptr(), s_w.data_ptr(), N, K,
+                                              Y.data_ptr(), _stream(Xq_tok)), "fp8q_moe_grouped_linear_gather")
     return Y
 
 

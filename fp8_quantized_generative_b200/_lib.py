@@ -58,6 +58,7 @@ SIGNATURES = {
     "fp8q_linear_fmt": (_INT, [_P, _INT, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "fp8q_moe_grouped_linear_fmt": (_INT, [_P, _INT, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_quantize_weight_blockwise": (_INT, [_P, _I32, _I64, _I64, _P, _P, _P]),
+    "fp8q_moe_grouped_linear_gather": (_INT, [_P, _P, _I64, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_moe_grouped_linear_blockscaled": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_e4m3_encode_f32": (_INT, [_P, _I64, _P, _P]),
     "fp8q_set_gemm_tuning": (_INT, [_INT, _INT, _INT]),
@@ -140,6 +141,11 @@ def fp8q_linear_fmt(Xq, x_fmt, s_x, Wq, s_w, M, N, K, Y, stream):
 
 def fp8q_moe_grouped_linear_fmt(Xq, x_fmt, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream):
     return lib().fp8q_moe_grouped_linear_fmt(Xq, x_fmt, s_x, offsets, E, rows, Wq, s_w, N, K, Y, stream)
+
+
+def fp8q_moe_grouped_linear_gather(Xq_tok, s_x_tok, tokens, row_token, offsets, E, rows, Wq, s_w, N, K, Y, stream):
+    return lib().fp8q_moe_grouped_linear_gather(Xq_tok, s_x_tok, tokens, row_token, offsets, E, rows, Wq, s_w, N, K,
+                                                Y, stream)
 
 
 def fp8q_quantize_weight_blockwise(W, E, N, K, Wq, s_wb, stream):

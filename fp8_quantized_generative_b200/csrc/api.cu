@@ -224,7 +224,7 @@ cudaError_t launch_ex(void (*kernel)(Args...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <bool kGrouped>
+template <bool kGrouped, bool kGather = false>
 fp8q_status launch_gemm(const uint8_t* A, int64_t a_rows, const uint8_t* B, int64_t b_rows, const GemmParams& p,
                         int64_t tiles_upper_bound, cudaStream_t st) {
   constexpr int BN = kGrouped ? kBNGrouped : kBN;
@@ -241,9 +241,9 @@ fp8q_status launch_gemm(const uint8_t* A, int64_t a_rows, const uint8_t* B, int6
   CUtensorMap ty;
   s = make_output_map(&ty, p.Y, p.rows, p.N);
   if (s != FP8Q_OK) return s;
-  auto kernel = fp8_gemm_kernel<BN, STAGES, kGrouped>;
+  auto kernel = fp8_gemm_kernel<BN, STAGES, kGrouped, kGather>;
   const size_t smem = L::smem_bytes(kGrouped ? p.E : 0);
-  e = ensure_smem<fp8_gemm_kernel<BN, STAGES, kGrouped>>(L::smem_bytes(kGrouped ? kMaxExperts : 0), dev);
+  e = ensure_smem<fp8_gemm_kernel<BN, STAGES, kGrouped, kGather>>(L::smem_bytes(kGrouped ? kMaxExperts : 0), dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   const int grid = static_cast<int>(tiles_upper_bound < sms ? (tiles_upper_bound < 1 ? 1 : tiles_upper_bound) : sms);
   e = launch_ex(kernel, dim3(grid), dim3(kGemmThreads), smem, st, 1, true, ta, tb, ty, p);
@@ -796,6 +796,39 @@ fp8q_status fp8q_moe_grouped_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, co
   }
   const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBNGrouped - 1) / kBNGrouped);
   return launch_gemm<true>(Xq, rows, Wq, int64_t(E) * N, p, tiles, static_cast<cudaStream_t>(stream));
+}
+
+fp8q_status fp8q_moe_grouped_linear_gather(const uint8_t* Xq_tok, const float* s_x_tok, int64_t tokens,
+                                           const int32_t* row_token, const int32_t* offsets, int32_t E, int64_t rows,
+                                           const uint8_t* Wq, const float* s_w, int64_t N, int64_t K, void* Y_f16,
+                                           void* stream) {
+  if (E < 1 || E > kMaxExperts) return invalid("E must be in [1, 1024]");
+  if (rows < 0 || rows > kMaxDim) return invalid("rows out of range");
+  if (tokens <= 0 || tokens > kMaxDim) return invalid("tokens must be positive");
+  if (N <= 0 || N % 8 != 0 || int64_t(E) * N > kMaxDim) return invalid("N must be positive, a multiple of 8, E*N < 2^31");
+  if (K <= 0 || K > kMaxDim || K % 16 != 0) return invalid("K must be positive and a multiple of 16");
+  if (offsets == nullptr || (reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return invalid("offsets pointer");
+  if (row_token == nullptr || (reinterpret_cast<uintptr_t>(row_token) & 3u) != 0) return invalid("row_token pointer");
+  if (rows == 0) return FP8Q_OK;
+  if (!aligned16(Xq_tok) || !aligned16(s_x_tok) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y_f16))
+    return invalid("null or non-16-byte-aligned pointer");
+  GemmParams p = {};   // every field set below; zero for the rest
+  p.s_x = s_x_tok;
+  p.s_w = s_w;
+  p.Y = static_cast<__half*>(Y_f16);
+  p.offsets = offsets;
+  p.rows = static_cast<int>(rows);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.E = E;
+  p.tail_q = 1;
+  p.x_fmt = FP8Q_FMT_E4M3;
+  p.xq = Xq_tok;
+  p.row_token = row_token;
+  p.tokens = static_cast<int>(tokens);
+  const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBNGrouped - 1) / kBNGrouped);
+  // the A tensor map (token matrix) is built but unused: the producer gathers the rows
+  return launch_gemm<true, true>(Xq_tok, tokens, Wq, int64_t(E) * N, p, tiles, static_cast<cudaStream_t>(stream));
 }
 
 fp8q_status fp8q_quantize_weight_blockwise(const void* W_f16, int32_t E, int64_t N, int64_t K, uint8_t* Wq,

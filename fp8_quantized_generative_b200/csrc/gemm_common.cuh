@@ -45,7 +45,19 @@ struct GemmParams {
   int l2_prefetch;          // split-K: 1 = prefetch the rest of the weight slice into L2 at start
   int half_tiles;           // CTA-pair grouped kernel: an expert's last <= 128 rows as an M = 128 pair tile
   int x_fmt;                // activation code format (Fp8Fmt): E4M3, or E5M2 for the variant
+  const uint8_t* xq;        // grouped gather: the token matrix of activation codes [tokens, K]
+  const int32_t* row_token; // grouped gather: row r of the product reads token row_token[r] (nullptr: row r)
+  int tokens;               // grouped gather: rows of the token matrix
 };
+
+// Row of the activation codes / scales that product row r reads (the row
+// itself, or its token in the gathered MoE form; an index out of range reads
+// row 0 and is reported by the producer).
+__device__ __forceinline__ int act_row(const GemmParams& p, int r) {
+  if (p.row_token == nullptr) return r;
+  const int t = __ldg(p.row_token + r);
+  return (t >= 0 && t < p.tokens) ? t : 0;
+}
 
 // One output slab of a CTA: 128 rows starting at row0, BN columns at n0.
 struct EpiTile {
@@ -112,7 +124,7 @@ __device__ __forceinline__ EpiScales<kMaxChunks> epilogue_scales(const EpiTile& 
                                                                  const EpiWarpView& w, int lane) {
   EpiScales<kMaxChunks> e;
   const int r = w.qrow0 + lane;
-  e.sx = r < t.row_end ? __ldg(p.s_x + r) : 0.0f;
+  e.sx = r < t.row_end ? __ldg(p.s_x + act_row(p, r)) : 0.0f;
 #pragma unroll
   for (int j = 0; j < kMaxChunks; ++j) {
     const int cl = w.col0 + j * 32 + lane;

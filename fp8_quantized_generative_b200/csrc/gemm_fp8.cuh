@@ -24,6 +24,15 @@
 // (no host synchronization): tiles are ordered (expert, n-block, m-block), so
 // the m-blocks that share one expert weight tile run back to back and reuse
 // it from L2.  No TMA multicast is used anywhere.
+//
+// Gather form (kGather, MoE): product row r reads activation row
+// row_token[r] of the token matrix (tokens quantized once; no permuted
+// copy).  The whole producer warp then fills a stage's A tile itself: each
+// lane copies four rows with 16-byte cp.async (zero-filled past K or past the
+// expert group) straight into the 128-byte-swizzled layout the MMA reads,
+// and once its copies of a stage have landed (one stage later, keeping
+// copies in flight) fences them for the async proxy and arrives on the
+// stage's barrier; the weight tile still comes by TMA.
 #pragma once
 
 #include "gemm_common.cuh"
@@ -90,12 +99,15 @@ __device__ __forceinline__ TileCoord decode_tile(int t, const GemmParams& p, int
   return c;
 }
 
-template <int BN, int STAGES, bool kGrouped>
+template <int BN, int STAGES, bool kGrouped, bool kGather = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
   using L = GemmLayout<BN, STAGES>;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  static_assert(!kGather || kGrouped, "gathered rows are a grouped (MoE) form");
+  constexpr int kGatherLag = 1;   // stages of row copies in flight before a stage is signalled
+  static_assert(!kGather || kGatherLag < STAGES, "lag");
   // A = activations: E4M3, or E5M2 for the activation-format variant
   const uint32_t kIdesc = idesc_e4m3_f32(kBM, BN) | idesc_a_fmt(p.x_fmt);
 
@@ -125,7 +137,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], kGather ? 33 : 1);   // gather: + one arrival per producer lane
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -177,7 +189,79 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // grid before touching anything this grid reads or writes).
   pdl_launch_dependents();
 
-  if (warp == 0) {
+  if (kGather && warp == 0) {
+    // ------------------------------------------------------------ producer (row gather, whole warp)
+    int s = 0, sig = 0, pending = 0;
+    uint32_t ph = 0, armed = 0, armed_ph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const TileCoord c = decode_tile<kGrouped, BN>(t, p, num_m, num_n, tile_prefix, offs);
+      int tok[4];   // tokens of this lane's rows lane, lane+32, lane+64, lane+96 (-1: zero row)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int row = c.a_row0 + lane + 32 * i;
+        tok[i] = row < c.row_end ? __ldg(p.row_token + row) : -1;
+        if (tok[i] >= p.tokens || (row < c.row_end && tok[i] < 0)) {
+          raise_error(0x8u);
+          tok[i] = -1;
+        }
+      }
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], L::kBBytes);
+          tma_load_2d(sB + s * L::kBBytes, &tmB, &full[s], kb * kBK, c.b_row0);
+        }
+        armed |= 1u << s;
+        armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
+        const uint32_t dst0 = smem_u32(sA + s * L::kABytes);
+        // one instruction copies 4 whole rows: lane l takes 16-byte chunk l % 8
+        // of row 4i + l / 8 (coalesced 128-byte lines); the row's token is
+        // held by lane (row % 32) in tok[row / 32]
+        const int ch = lane & 7;
+        const int k = kb * kBK + ch * 16;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int r = 4 * i + (lane >> 3);
+          const int tk = __shfl_sync(0xffffffffu, tok[i >> 3], r & 31);
+          const bool v = tk >= 0 && k < p.K;
+          const uint8_t* src = p.xq + (v ? static_cast<int64_t>(tk) * p.K + k : 0);
+          cp_async_16_zfill(dst0 + static_cast<uint32_t>(r * kBK + ((ch ^ (r & 7)) << 4)), src, v ? 16u : 0u);
+        }
+        cp_async_commit();
+        if (++pending > kGatherLag) {
+          // the copies of stage `sig` have landed: hand them to the async proxy and signal
+          cp_async_wait_group<kGatherLag>();
+          fence_proxy_async_smem();
+          mbar_arrive(&full[sig]);
+          if (++sig == STAGES) sig = 0;
+          --pending;
+        }
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    cp_async_wait_group<0>();
+    fence_proxy_async_smem();
+    for (; pending > 0; --pending) {
+      mbar_arrive(&full[sig]);
+      if (++sig == STAGES) sig = 0;
+    }
+    if (!ok) {
+      raise_error(0x1u);
+      *abort_flag = 1;
+    }
+    // No weight copy may still be in flight when the CTA exits.
+    if (lane == 0)
+      for (int i = 0; i < STAGES; ++i)
+        if (armed & (1u << i)) mbar_wait(&full[i], (armed_ph >> i) & 1u, nullptr);
+    __syncwarp();
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int s = 0;

@@ -325,6 +325,18 @@ __device__ __forceinline__ void mma_commit_pair_mc(uint64_t* bar, uint16_t cta_m
       : "memory");
 }
 
+// ---------------------------------------------------------------- cp.async (row gathers)
+// 16-byte global -> shared copy; src_bytes < 16 zero-fills the rest (0: all zero, src not read).
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t smem_dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// All but the N most recent cp.async groups of this thread have completed.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---------------------------------------------------------------- PDL
 // Programmatic dependent launch: a dependent grid may start once every CTA
 // of this grid has called launch_dependents (or exited); the dependent waits

@@ -245,6 +245,22 @@ fp8q_status fp8q_moe_grouped_linear_blockscaled(const uint8_t* Xq, const float* 
                                                 int64_t N, int64_t K,
                                                 void* Y_f16, void* stream);
 
+/*
+ * MoE expert grouped linear reading its rows straight from the token matrix
+ * [P1 关键证据 item 2 (sparse MoE); P2 §3.2 (expert pipeline)]: the
+ * activations are quantized once per token (Xq_tok [tokens,K] uint8, s_x_tok
+ * [tokens] fp32, from fp8q_quantize_rows_dynamic), and row r of the grouped
+ * product (rows in expert order, offsets as for fp8q_moe_grouped_linear)
+ * reads token row_token[r] (int32 [rows], device).  Same result as
+ * fp8q_moe_grouped_linear on the gathered rows, without the gathered copy.
+ * Y_f16 [rows,N].  A row_token entry outside [0, tokens) sets
+ * FP8Q_DEVERR_BAD_OFFSETS and that row reads zeros.
+ */
+fp8q_status fp8q_moe_grouped_linear_gather(const uint8_t* Xq_tok, const float* s_x_tok, int64_t tokens,
+                                           const int32_t* row_token, const int32_t* offsets, int32_t E,
+                                           int64_t rows, const uint8_t* Wq, const float* s_w,
+                                           int64_t N, int64_t K, void* Y_f16, void* stream);
+
 /* fp8q_moe_grouped_linear with the activation codes Xq in format x_fmt. */
 fp8q_status fp8q_moe_grouped_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, const float* s_x,
                                         const int32_t* offsets, int32_t E, int64_t rows,

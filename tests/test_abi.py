@@ -158,3 +158,15 @@ def test_blockscaled_rejects(L):
     assert mo(a, a, 0x1002, 4, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG  # offsets alignment
     assert mo(a, a, a, 4, 8, a, BAD, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
     assert mo(0, 0, a, 4, 0, 0, 0, 16, 32, 0, 0) == _lib.FP8Q_OK                    # no rows
+
+
+def test_gather_rejects(L):
+    a = 0x1000
+    g = _lib.fp8q_moe_grouped_linear_gather
+    assert g(a, a, 0, a, a, 4, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG      # no tokens
+    assert g(a, a, 10, 0, a, 4, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG     # null row_token
+    assert g(a, a, 10, 0x1002, a, 4, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert g(a, a, 10, a, a, 0, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert g(a, a, 10, a, a, 4, 8, a, a, 12, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert g(BAD, a, 10, a, a, 4, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert g(0, 0, 10, a, a, 4, 0, 0, 0, 16, 32, 0, 0) == _lib.FP8Q_OK                  # no rows

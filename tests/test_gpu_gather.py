@@ -1,0 +1,103 @@
+"""GPU parity of the MoE grouped linear that reads its rows from the token
+matrix (fp8q_moe_grouped_linear_gather): tokens quantized once, row r of the
+grouped product reads token row_token[r] (the FP16 top-2 router's grouping).
+Outputs within the path's tolerance of oracle.moe_gather_ref, and equal to
+the grouped linear on a gathered copy.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_gather_ref, quant_rows
+from fp8_quantized_generative_b200 import workloads as wl
+
+from parity import assert_close_f16, assert_no_device_error, sample_rows, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fq():
+    import fp8_quantized_generative_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def routed(T, E, seed):
+    logits = wl.random_f16((T, E), seed=seed).numpy()
+    row_token, offsets = wl.group_by_expert(wl.route_top2(logits), E)
+    return row_token.astype(np.int32), np.asarray(offsets, dtype=np.int32)
+
+
+def run_gather(fq, X, row_token, offsets, W):
+    Xq, s_x = fq.quantize_rows_dynamic(X.cuda())
+    Wq, s_w = fq.quantize_weight_per_channel(W.cuda())
+    Y = torch.full((len(row_token), W.shape[1]), float("nan"), dtype=torch.float16, device="cuda")
+    fq.moe_grouped_linear_gather(Xq, s_x, torch.from_numpy(row_token).cuda(), torch.from_numpy(offsets).cuda(),
+                                 Wq, s_w, out=Y)
+    torch.cuda.synchronize()
+    return Y, (Xq, s_x, Wq, s_w)
+
+
+def oracle_gather(X, row_token, offsets, W, rows=None):
+    E, N, K = W.shape
+    xq, sx = quant_rows(X.numpy())
+    q = [quant_rows(W[e].numpy()) for e in range(E)]
+    Wq = np.stack([c for c, _ in q])
+    sw = np.stack([s for _, s in q])
+    ref = moe_gather_ref(xq, sx, row_token, offsets, Wq, sw)
+    return ref if rows is None else ref[rows]
+
+
+@pytest.mark.parametrize("T,E,N,K", [(40, 6, 264, 272), (300, 8, 256, 512), (1, 3, 64, 128)])
+def test_routed_small(fq, T, E, N, K):
+    row_token, offsets = routed(T, E, seed=T + E)
+    X = wl.random_f16((T, K), seed=T * 3 + 1)
+    W = wl.random_f16((E, N, K), seed=E * 5 + 2, std=0.02)
+    Y, _ = run_gather(fq, X, row_token, offsets, W)
+    assert_close_f16(to_np(Y), oracle_gather(X, row_token, offsets, W), f"gather T={T} E={E}")
+    assert_no_device_error()
+
+
+def test_equals_grouped_linear_on_gathered_copy(fq):
+    T, E, N, K = 500, 10, 512, 1024
+    row_token, offsets = routed(T, E, seed=9)
+    X = wl.random_f16((T, K), seed=10)
+    W = wl.random_f16((E, N, K), seed=11, std=0.02)
+    Y, (Xq, s_x, Wq, s_w) = run_gather(fq, X, row_token, offsets, W)
+    idx = torch.from_numpy(row_token.astype(np.int64)).cuda()
+    Y2 = fq.moe_grouped_linear(Xq[idx].contiguous(), s_x[idx].contiguous(), torch.from_numpy(offsets).cuda(), Wq, s_w)
+    torch.cuda.synchronize()
+    # same codes, scales, tiles and accumulation order: bitwise equal
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_bad_token_index_is_reported(fq):
+    T, E, N, K = 8, 2, 64, 128
+    X = wl.random_f16((T, K), seed=3).cuda()
+    Xq, s_x = fq.quantize_rows_dynamic(X)
+    Wq, s_w = fq.quantize_weight_per_channel(wl.random_f16((E, N, K), seed=4, std=0.02).cuda())
+    row_token = torch.tensor([0, 1, 2, 9, 4, 5], dtype=torch.int32, device="cuda")      # 9 >= T
+    offsets = torch.tensor([0, 3, 6], dtype=torch.int32, device="cuda")
+    fq.moe_grouped_linear_gather(Xq, s_x, row_token, offsets, Wq, s_w)
+    assert fq.device_error() == 0x8
+
+
+def test_moe_up_from_tokens(fq):
+    m = wl.moe()
+    row_token = np.asarray(m.token_of_row, dtype=np.int32)
+    offsets = np.asarray(m.offsets, dtype=np.int32)
+    Y, _ = run_gather(fq, m.X, row_token, offsets, m.W_up)
+    rows = sample_rows(len(row_token), 256, seed=12)
+    E, N, K = m.W_up.shape
+    # oracle on the sampled rows only (quantize the sampled tokens; each row with its expert)
+    expert_of = np.searchsorted(offsets.astype(np.int64), rows, side="right") - 1
+    xq, sx = quant_rows(m.X.numpy()[row_token[rows]])
+    ref = np.zeros((len(rows), N), np.float16)
+    from oracle import linear_ref
+    for e in np.unique(expert_of):
+        sel = expert_of == e
+        wq, sw = quant_rows(m.W_up[e].numpy())
+        ref[sel] = linear_ref(xq[sel], sx[sel], wq, sw)
+    assert_close_f16(to_np(Y)[rows], ref, "moe up from tokens")
+    assert_no_device_error()

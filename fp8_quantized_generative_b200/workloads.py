@@ -127,6 +127,13 @@ def route_top2(logits_f16: np.ndarray, topk: int = MOE_TOPK) -> np.ndarray:
     return np.argsort(neg, axis=1, kind="stable")[:, :topk].astype(np.int64)
 
 
+def _expert_order(experts: np.ndarray) -> np.ndarray:
+    """Permutation of the flattened (token, slot) pairs that sorts them by (expert, token)."""
+    T, k = experts.shape
+    tok = np.repeat(np.arange(T, dtype=np.int64), k)
+    return np.lexsort((tok, experts.reshape(-1)))
+
+
 def group_by_expert(experts: np.ndarray, n_experts: int) -> tuple[np.ndarray, np.ndarray]:
     """Order (token, slot) pairs by (expert, token).
 
@@ -135,12 +142,25 @@ def group_by_expert(experts: np.ndarray, n_experts: int) -> tuple[np.ndarray, np
     """
     T, k = experts.shape
     tok = np.repeat(np.arange(T, dtype=np.int64), k)
-    exp = experts.reshape(-1)
-    order = np.lexsort((tok, exp))
-    counts = np.bincount(exp, minlength=n_experts)
+    order = _expert_order(experts)
+    counts = np.bincount(experts.reshape(-1), minlength=n_experts)
     offsets = np.zeros(n_experts + 1, dtype=np.int64)
     np.cumsum(counts, out=offsets[1:])
     return tok[order], offsets.astype(np.int32)
+
+
+def gate_weights(logits_f16: np.ndarray, experts: np.ndarray) -> np.ndarray:
+    """Combine weights of each token's selected experts: a softmax over the
+    selected FP16 logits, in float32 (harness side of the router; the pages
+    fix no combine rule).  Returns float32 [T, topk], rows summing to ~1."""
+    sel = np.take_along_axis(logits_f16.astype(np.float32), experts, axis=1)
+    z = np.exp(sel - sel.max(axis=1, keepdims=True), dtype=np.float32)
+    return (z / z.sum(axis=1, keepdims=True)).astype(np.float32)
+
+
+def row_weights(weights: np.ndarray, experts: np.ndarray) -> np.ndarray:
+    """The combine weight of every grouped row (same order as group_by_expert): float32 [T*topk]."""
+    return weights.reshape(-1)[_expert_order(experts)].astype(np.float32)
 
 
 @dataclass
@@ -152,6 +172,7 @@ class MoE:
     X_perm: torch.Tensor     # fp16 [T*topk, d] rows in expert order
     W_up: torch.Tensor       # fp16 [E, F, d]
     W_down: torch.Tensor     # fp16 [E, d, F]
+    row_weight: np.ndarray   # float32 [T*topk] combine weight of each grouped row (see gate_weights)
 
 
 def moe(T: int = MOE_T, d: int = MOE_D, E: int = MOE_E, F: int = MOE_F,
@@ -167,7 +188,8 @@ def moe(T: int = MOE_T, d: int = MOE_D, E: int = MOE_E, F: int = MOE_F,
         W_down = normal_f16((E, d, F), W_STD, gw)
     else:
         W_up = W_down = None
-    return MoE(X, logits, token_of_row, offsets, X_perm, W_up, W_down)
+    row_weight = row_weights(gate_weights(logits.numpy(), experts), experts)
+    return MoE(X, logits, token_of_row, offsets, X_perm, W_up, W_down, row_weight)
 
 
 def offsets_from_counts(counts) -> np.ndarray:

@@ -28,9 +28,10 @@ rows, a library cast routine and brute force; none is "parity unpinned".
 from .e4m3 import E4M3_MAX, e4m3_decode, e4m3_encode
 from .e5m2 import E5M2_MAX, e5m2_decode, e5m2_encode
 from .quant import EPS, quant_blocks, quant_rows, quant_tensor
-from .linear import (linear_blockscaled_ref, linear_f64_unquantized, linear_ref, moe_blockscaled_ref, moe_gather_ref,
-                     moe_ref)
+from .linear import (linear_blockscaled_ref, linear_f64_unquantized, linear_ref, moe_blockscaled_ref, moe_combine_ref,
+                     moe_gather_ref, moe_ref)
 
 __all__ = ["E4M3_MAX", "e4m3_decode", "e4m3_encode", "E5M2_MAX", "e5m2_decode", "e5m2_encode",
            "EPS", "quant_rows", "quant_tensor", "quant_blocks", "linear_ref", "moe_ref",
-           "linear_blockscaled_ref", "moe_blockscaled_ref", "moe_gather_ref", "linear_f64_unquantized"]
+           "linear_blockscaled_ref", "moe_blockscaled_ref", "moe_gather_ref", "moe_combine_ref",
+           "linear_f64_unquantized"]

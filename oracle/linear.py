@@ -35,13 +35,17 @@ from .e5m2 import e5m2_decode
 _DECODERS = {"e4m3": e4m3_decode, "e5m2": e5m2_decode}
 
 
-def linear_ref(Xq, s_x, Wq, s_w, x_fmt: str = "e4m3") -> np.ndarray:
-    """Xq uint8 [M,K], s_x f32 [M], Wq uint8 [N,K], s_w f32 [N] -> float16 [M,N]."""
+def _linear_f64(Xq, s_x, Wq, s_w, x_fmt: str = "e4m3") -> np.ndarray:
+    """The dequantized product (P * s_x) * s_w in float64, before the fp16 cast."""
     Dx = _DECODERS[x_fmt](Xq)
     Dw = e4m3_decode(Wq)
     P = Dx @ Dw.T
-    Y = (P * np.asarray(s_x, dtype=np.float64)[:, None]) * np.asarray(s_w, dtype=np.float64)[None, :]
-    return Y.astype(np.float16)
+    return (P * np.asarray(s_x, dtype=np.float64)[:, None]) * np.asarray(s_w, dtype=np.float64)[None, :]
+
+
+def linear_ref(Xq, s_x, Wq, s_w, x_fmt: str = "e4m3") -> np.ndarray:
+    """Xq uint8 [M,K], s_x f32 [M], Wq uint8 [N,K], s_w f32 [N] -> float16 [M,N]."""
+    return _linear_f64(Xq, s_x, Wq, s_w, x_fmt).astype(np.float16)
 
 
 def moe_ref(Xq, s_x, offsets, Wq, s_w, x_fmt: str = "e4m3") -> np.ndarray:
@@ -114,3 +118,38 @@ def moe_gather_ref(Xq_tok, s_x_tok, row_token, offsets, Wq, s_w) -> np.ndarray:
     if row_token.size and (row_token.min() < 0 or row_token.max() >= Xq_tok.shape[0]):
         raise ValueError("row_token out of range")
     return moe_ref(Xq_tok[row_token], np.asarray(s_x_tok)[row_token], offsets, Wq, s_w)
+
+
+def moe_combine_ref(Xq, s_x, offsets, Wq, s_w, row_token, row_weight, tokens: int) -> np.ndarray:
+    """Grouped linear whose rows are combined back into their tokens.
+
+    The down projection of the MoE layer with the top-k combine in its
+    epilogue [P1 关键证据 item 2; P2 §3.2]: each grouped row r (expert order,
+    offsets as in moe_ref) yields y[r] = (P * s_x) * s_w in float64, its
+    contribution c[r] = fp16(row_weight[r] * y[r]) (one rounding), and the
+    output row of token t is the FP16 scatter-add of its contributions:
+    out[t] starts at 0 and each contribution is added with one fp16 rounding
+    of the exact sum.  With two rows per token (top-2) the result does not
+    depend on the order of the additions (0 + a = a exactly and fp16
+    addition is commutative).  Returns float16 [tokens, N].
+    """
+    offsets = np.asarray(offsets, dtype=np.int64)
+    E, N, _ = np.asarray(Wq).shape
+    R = np.asarray(Xq).shape[0]
+    row_token = np.asarray(row_token, dtype=np.int64)
+    w = np.asarray(row_weight, dtype=np.float32).astype(np.float64)
+    if offsets.shape != (E + 1,) or offsets[0] != 0 or offsets[-1] != R or np.any(np.diff(offsets) < 0):
+        raise ValueError("offsets must be non-decreasing, start at 0 and end at the row count")
+    if row_token.shape != (R,) or (R and (row_token.min() < 0 or row_token.max() >= tokens)):
+        raise ValueError("row_token out of range")
+    out = np.zeros((tokens, N), dtype=np.float16)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        y = _linear_f64(Xq[lo:hi], s_x[lo:hi], Wq[e], s_w[e])
+        c = (w[lo:hi, None] * y).astype(np.float16)
+        for i, r in enumerate(range(lo, hi)):
+            t = row_token[r]
+            out[t] = (out[t].astype(np.float64) + c[i].astype(np.float64)).astype(np.float16)
+    return out

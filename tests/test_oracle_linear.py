@@ -252,3 +252,69 @@ def test_moe_gather_matches_permuted_rows_and_identity():
                                   moe_ref(xq_p, sx_p, offsets, Wq, sw).view(np.uint16))
     with pytest.raises(ValueError):
         moe_gather_ref(xq, sx, np.array([0, T]), np.array([0, 2]), Wq[:1], sw[:1])
+
+
+# ---------------------------------------------------------------------------
+# Top-k combine in the down projection's epilogue (FP16 scatter-add).
+
+def _moe_setup(seed, T=30, E=5, N=16, K=48):
+    from fp8_quantized_generative_b200 import workloads as wl
+    rng = np.random.default_rng(seed)
+    logits = rng.standard_normal((T, E)).astype(np.float16)
+    experts = wl.route_top2(logits)
+    row_token, offsets = wl.group_by_expert(experts, E)
+    row_w = wl.row_weights(wl.gate_weights(logits, experts), experts)
+    H = rng.standard_normal((len(row_token), K)).astype(np.float16)
+    W = (rng.standard_normal((E, N, K)) * 0.05).astype(np.float16)
+    hq, sh = quant_rows(H)
+    q = [quant_rows(W[e]) for e in range(E)]
+    Wq = np.stack([c for c, _ in q]); sw = np.stack([s for _, s in q])
+    return T, row_token, offsets, row_w, hq, sh, Wq, sw
+
+
+def test_combine_with_one_hot_weights_returns_the_rows():
+    from oracle import moe_combine_ref
+    T, row_token, offsets, _, hq, sh, Wq, sw = _moe_setup(71)
+    # weight 1 on each token's first row, 0 on the other: the output is that row of moe_ref
+    first = np.zeros(len(row_token), np.float32)
+    seen = set()
+    for r in np.argsort(row_token, kind="stable"):
+        if row_token[r] not in seen:
+            first[r] = 1.0
+            seen.add(row_token[r])
+    out = moe_combine_ref(hq, sh, offsets, Wq, sw, row_token, first, T)
+    Y = moe_ref(hq, sh, offsets, Wq, sw)
+    for r in np.nonzero(first)[0]:
+        np.testing.assert_array_equal(out[row_token[r]].view(np.uint16), Y[r].view(np.uint16))
+
+
+def test_combine_matches_an_explicit_per_token_loop():
+    from oracle import moe_combine_ref
+    T, row_token, offsets, row_w, hq, sh, Wq, sw = _moe_setup(73)
+    out = moe_combine_ref(hq, sh, offsets, Wq, sw, row_token, row_w, T)
+    # restatement: y of every row from unquantized-arithmetic building blocks, then per token
+    E = Wq.shape[0]
+    expert_of = np.searchsorted(offsets.astype(np.int64), np.arange(len(row_token)), side="right") - 1
+    for t in range(T):
+        rows = np.nonzero(row_token == t)[0]
+        assert len(rows) == 2
+        acc = np.float16(0.0)
+        for r in rows:
+            e = expert_of[r]
+            yv = (e4m3_decode(hq[r])[None, :] @ e4m3_decode(Wq[e]).T)[0] * np.float64(sh[r]) * sw[e].astype(np.float64)
+            c = (np.float64(row_w[r]) * yv).astype(np.float16)
+            acc = (np.asarray(acc, np.float64) + c.astype(np.float64)).astype(np.float16)
+        np.testing.assert_array_equal(out[t].view(np.uint16), np.asarray(acc).view(np.uint16))
+
+
+def test_combine_is_within_fp16_rounding_of_the_weighted_sum():
+    from oracle import moe_combine_ref
+    T, row_token, offsets, row_w, hq, sh, Wq, sw = _moe_setup(79, T=64, E=6, N=32, K=64)
+    out = moe_combine_ref(hq, sh, offsets, Wq, sw, row_token, row_w, T).astype(np.float64)
+    Y = moe_ref(hq, sh, offsets, Wq, sw)   # fp16 rows
+    exact = np.zeros_like(out)
+    mag = np.zeros_like(out)
+    np.add.at(exact, row_token, row_w[:, None].astype(np.float64) * Y.astype(np.float64))
+    np.add.at(mag, row_token, np.abs(row_w[:, None].astype(np.float64) * Y.astype(np.float64)))
+    # three fp16 roundings (each row's y, each contribution, the sum): <= 2^-10 of the magnitudes
+    assert np.all(np.abs(out - exact) <= 2.0 ** -10 * (mag + np.abs(exact)) + 2.0 ** -24)

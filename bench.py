@@ -74,11 +74,14 @@ def workload_spec(name: str):
         return ("moe_ffn T=8192 top2 E=64 d=2048 F=1024 (16384 grouped rows)", "moe",
                 (m.X_perm, m.offsets, m.W_up, m.W_down))
     if name == "moe_tokens":
-        # the same layer from the token matrix: tokens quantized once, the up
-        # projection gathers its rows by the router's grouping
+        # the same layer from and back to the token matrix: tokens quantized
+        # once, the up projection gathers its rows by the router's grouping and
+        # the down projection adds each row, weighted, into its token (combine)
         m = wl.moe()
-        return ("moe_ffn T=8192 top2 E=64 d=2048 F=1024 from the 8192-token matrix (row gather)", "moe",
-                (m.X, m.offsets, m.W_up, m.W_down, np.asarray(m.token_of_row, dtype=np.int32)))
+        return ("moe_ffn T=8192 top2 E=64 d=2048 F=1024 from and back to the 8192-token matrix "
+                "(dispatch to the expert rows, weighted top-2 combine)", "moe",
+                (m.X, m.offsets, m.W_up, m.W_down, np.asarray(m.token_of_row, dtype=np.int32),
+                 np.asarray(m.row_weight, dtype=np.float32)))
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -145,7 +148,8 @@ class ClockSampler:
 class Plan:
     """Device buffers (rotated sets) and the raw C-ABI launch sequence of one step."""
 
-    def __init__(self, kind, tensors, device, min_rotation_bytes, fused=True, x_fmt="e4m3", weights="channel"):
+    def __init__(self, kind, tensors, device, min_rotation_bytes, fused=True, x_fmt="e4m3", weights="channel",
+                 dispatch="quant"):
         import fp8_quantized_generative_b200 as fq
         from fp8_quantized_generative_b200 import _lib
         self.fq, self.L = fq, _lib
@@ -157,6 +161,8 @@ class Plan:
         if (weights == "tensor" and kind != "dense") or (weights == "block" and kind == "dense"):
             raise SystemExit(f"--weight-scales {weights} applies to "
                              f"{'dense' if weights == 'tensor' else 'moe'} workloads only")
+        if kind != "dense" and len(tensors) > 4 and (weights != "channel" or x_fmt != "e4m3"):
+            raise SystemExit("the row-gather / combine MoE form runs E4M3 activations with per-channel weights")
         self.weights = weights
         self.fmt = _lib.FORMATS[x_fmt]
         # Up to 16 token rows the library quantizes inside the GEMM (one launch; E4M3 only).
@@ -171,13 +177,18 @@ class Plan:
             Xp, offsets, Wu, Wd = tensors[:4]
             # gather form: Xp is the token matrix and tensors[4] the row -> token map
             self.row_token = tensors[4] if len(tensors) > 4 else None
+            self.row_weight = tensors[5] if len(tensors) > 5 else None   # and the combine weights
+            # token -> grouped rows by the quantizer's store (quant), or grouped rows <- tokens by the GEMM (gemm)
+            self.dispatch = dispatch if self.row_token is not None else None
+            self.gather = self.dispatch == "gemm"
             self.T = Xp.shape[0]
             self.R = int(offsets[-1])
             self.D = Xp.shape[1]
             self.E, self.F, _ = Wu.shape
             self.flops = 2.0 * self.R * self.F * self.D * 2
+            self.out_rows = self.T if self.row_weight is not None else self.R
             per_set = (self.T * self.D * 3 + 8 * self.R + 2 * self.E * self.F * self.D + 8 * self.E * self.F
-                       + self.R * self.F * 5 + self.R * self.D * 2)
+                       + self.R * self.F * 5 + self.out_rows * self.D * 2 + 4 * self.R)
         self.sets = max(2, math.ceil(min_rotation_bytes / per_set))
         self.bufs = []
         for i in range(self.sets):
@@ -194,15 +205,20 @@ class Plan:
                 b["off"] = torch.from_numpy(offsets).to(device)
                 if self.row_token is not None:
                     b["rt"] = torch.from_numpy(self.row_token).to(device)
+                if self.dispatch == "quant":
+                    b["tr"] = torch.from_numpy(wl.token_rows(self.row_token, self.T)).to(device)
+                if self.row_weight is not None:
+                    b["rw"] = torch.from_numpy(self.row_weight).to(device)
                 qw = fq.quantize_weight_blockwise if weights == "block" else fq.quantize_weight_per_channel
                 b["Wuq"], b["swu"] = qw(Wu.to(device))
                 b["Wdq"], b["swd"] = qw(Wd.to(device))
-                b["Xq"] = torch.empty((self.T, self.D), dtype=torch.uint8, device=device)
-                b["sx"] = torch.empty((self.T,), dtype=torch.float32, device=device)
+                xrows = self.R if self.dispatch == "quant" else self.T   # quantized rows: grouped or tokens
+                b["Xq"] = torch.empty((xrows, self.D), dtype=torch.uint8, device=device)
+                b["sx"] = torch.empty((xrows,), dtype=torch.float32, device=device)
                 b["H"] = torch.empty((self.R, self.F), dtype=torch.float16, device=device)
                 b["Hq"] = torch.empty((self.R, self.F), dtype=torch.uint8, device=device)
                 b["sh"] = torch.empty((self.R,), dtype=torch.float32, device=device)
-                b["Y"] = torch.empty((self.R, self.D), dtype=torch.float16, device=device)
+                b["Y"] = torch.empty((self.out_rows, self.D), dtype=torch.float16, device=device)
             b = {k: v for k, v in b.items()}
             b["p"] = {k: v.data_ptr() for k, v in b.items()}
             self.bufs.append(b)
@@ -216,8 +232,10 @@ class Plan:
             return ["fp8_quantized_linear_fused"]
         if self.kind == "dense":
             return ["quant_rows", "fp8_gemm"]
-        up = "fp8_grouped_gemm_up_gather" if self.row_token is not None else "fp8_grouped_gemm_up"
-        return ["quant_rows", up, "quant_rows_h", "fp8_grouped_gemm_down"]
+        up = "fp8_grouped_gemm_up_gather" if self.gather else "fp8_grouped_gemm_up"
+        down = "fp8_grouped_gemm_down_combine" if self.row_weight is not None else "fp8_grouped_gemm_down"
+        quant = "quant_rows_dispatch" if self.dispatch == "quant" else "quant_rows"
+        return [quant, up, "quant_rows_h", down]
 
     def kernel_bytes_flops(self):
         """Algorithmic bytes and FLOPs of each launch of one step."""
@@ -233,10 +251,15 @@ class Plan:
             su, sd = 4 * E * (-(-F // 128)) * (-(-D // 128)), 4 * E * (-(-D // 128)) * (-(-F // 128))
         else:
             su, sd = 4 * E * F, 4 * E * D
-        return [(self.T * D * 3 + 4 * self.T, 0.0),
+        # dispatch: each token read once and written to its grouped rows (+ the token -> row map)
+        q0 = ((self.T * D * 2 + R * D + 4 * R + 4 * self.T * 2, 0.0) if self.dispatch == "quant"
+              else (self.T * D * 3 + 4 * self.T, 0.0))
+        return [q0,
                 (R * D + E * F * D + 4 * R + su + 2 * R * F, 2.0 * R * F * D),
                 (R * F * 3 + 4 * R, 0.0),
-                (R * F + E * D * F + 4 * R + sd + 2 * R * D, 2.0 * R * D * F)]
+                (R * F + E * D * F + 4 * R + sd + 2 * R * D, 2.0 * R * D * F) if self.row_weight is None else
+                # combine: + token index and weight per row; the output is the [T, D] token matrix
+                (R * F + E * D * F + 12 * R + sd + 2 * self.T * D, 2.0 * R * D * F)]
 
     def launch(self, i, k):
         """Launch kernel k of step i (raw C ABI, integer pointers)."""
@@ -251,9 +274,12 @@ class Plan:
                 s = L.fp8q_linear_fmt(p["Xq"], self.fmt, p["sx"], p["Wq"], p["sw"], self.M, self.N, self.K, p["Y"],
                                       st)
         else:
-            if k == 0:
+            if k == 0 and self.dispatch == "quant":
+                s = L.fp8q_quantize_rows_dispatch(p["X"], self.T, self.D, self.fmt, p["tr"], 2, self.R, p["Xq"],
+                                                  p["sx"], st)
+            elif k == 0:
                 s = L.fp8q_quantize_rows_dynamic_fmt(p["X"], self.T, self.D, self.fmt, p["Xq"], p["sx"], st)
-            elif k == 1 and self.row_token is not None:
+            elif k == 1 and self.gather:
                 s = L.fp8q_moe_grouped_linear_gather(p["Xq"], p["sx"], self.T, p["rt"], p["off"], self.E, self.R,
                                                      p["Wuq"], p["swu"], self.F, self.D, p["H"], st)
             elif k == 1:
@@ -265,6 +291,9 @@ class Plan:
                                                       p["Wuq"], p["swu"], self.F, self.D, p["H"], st)
             elif k == 2:
                 s = L.fp8q_quantize_rows_dynamic_fmt(p["H"], self.R, self.F, self.fmt, p["Hq"], p["sh"], st)
+            elif self.row_weight is not None:
+                s = L.fp8q_moe_grouped_linear_combine(p["Hq"], p["sh"], p["off"], self.E, self.R, p["Wdq"], p["swd"],
+                                                      self.D, self.F, p["rt"], p["rw"], self.T, p["Y"], st)
             elif self.weights == "block":
                 s = L.fp8q_moe_grouped_linear_blockscaled(p["Hq"], p["sh"], p["off"], self.E, self.R, p["Wdq"],
                                                           p["swd"], self.D, self.F, p["Y"], st)
@@ -357,7 +386,7 @@ def timed_e2e(plan, tensors, steps):
     dev = plan.device
     main = torch.cuda.current_stream(dev)
     streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
-    out_shape = (plan.M, plan.N) if plan.kind == "dense" else (plan.R, plan.D)
+    out_shape = (plan.M, plan.N) if plan.kind == "dense" else (plan.out_rows, plan.D)
     xh = tensors[0].pin_memory()
     yh = [torch.empty(out_shape, dtype=torch.float16).pin_memory() for _ in range(2)]
     h2d, d2h = xh.numel() * 2, yh[0].numel() * 2
@@ -392,7 +421,7 @@ def timed_e2e(plan, tensors, steps):
 # --------------------------------------------------------------------------- oracle arm
 def oracle_sampler(kind, tensors, m_rows, n_rows, x_fmt="e4m3", weights="channel"):
     """A callable running the oracle on an (m_rows x n_rows) output sample; returns its FLOPs."""
-    from oracle import linear_blockscaled_ref, linear_ref, quant_blocks, quant_rows, quant_tensor
+    from oracle import linear_blockscaled_ref, linear_ref, moe_combine_ref, quant_blocks, quant_rows, quant_tensor
     if kind == "dense":
         X, W = tensors
         Xn = X.numpy()
@@ -434,14 +463,28 @@ def oracle_sampler(kind, tensors, m_rows, n_rows, x_fmt="e4m3", weights="channel
     Wuq, swu = quant_rows(Wu[e].numpy()[:n_rows])
     Wdq, swd = quant_rows(Wd[e].numpy()[:, :])
 
+    if len(tensors) > 5:
+        # combine form: the down projection adds each weighted row into its token
+        # (one row per token within one expert, so the sample's tokens are local)
+        rw = np.asarray(tensors[5][lo:lo + cnt], dtype=np.float32)
+        one = np.array([0, cnt], dtype=np.int64)
+        local = np.arange(cnt)
+
+        def down(hq, sh):
+            moe_combine_ref(hq, sh, one, Wdq[None, :n_rows, :hq.shape[1]], swd[None, :n_rows], local, rw, cnt)
+    else:
+        def down(hq, sh):
+            # down projection restricted to the sampled hidden columns
+            linear_ref(hq, sh, Wdq[:n_rows, :hq.shape[1]], swd[:n_rows], x_fmt)
+
     def run():
         xq, sx = quant_rows(Xn, x_fmt)
         h = linear_ref(xq, sx, Wuq, swu, x_fmt)
         hq, sh = quant_rows(h, x_fmt)
-        # down projection restricted to the sampled hidden columns
-        linear_ref(hq, sh, Wdq[:n_rows, :hq.shape[1]], swd[:n_rows], x_fmt)
+        down(hq, sh)
         return 2.0 * cnt * Wuq.shape[0] * D + 2.0 * cnt * n_rows * hq.shape[1]
-    return run, f"expert {e}: {cnt} rows through up ({n_rows} channels) and down ({n_rows} channels)"
+    return run, (f"expert {e}: {cnt} rows through up ({n_rows} channels) and down ({n_rows} channels)"
+                 + (", weighted combine into the rows' tokens" if len(tensors) > 5 else ""))
 
 
 def blas_threads():
@@ -541,6 +584,7 @@ def run_ours(args, world, rank, local):
     import fp8_quantized_generative_b200 as fq
     fq.set_gemm_tuning({"auto": 0, "single": 1, "pair": 2, "splitk": 3}[args.gemm], args.bn, args.ksplit)
     plan = Plan(kind, tensors, device, min_rotation_bytes=3 * L2_BYTES, fused=args.fused, x_fmt=args.x_fmt,
+                dispatch=args.dispatch,
                 weights=args.weight_scales)
     peaks, peak_src = load_peaks()
 
@@ -661,6 +705,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="qkv")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dispatch", default="quant", choices=["quant", "gemm"],
+                    help="moe_tokens: tokens reach their expert-grouped rows through the quantizer's store "
+                         "(quant) or through the up GEMM's row gather (gemm)")
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of a CUDA graph")
     ap.add_argument("--x-fmt", default="e4m3", choices=["e4m3", "e5m2"],
                     help="activation code format (e5m2: the pages' activation-format variant)")

@@ -27,6 +27,7 @@ from ._lib import Fp8qError, check, lib
 __all__ = [
     "Fp8qError", "lib", "quantize_rows_dynamic", "quantize_weight_per_channel", "quantize_weight_per_tensor",
     "quantize_weight_blockwise", "linear", "moe_grouped_linear", "moe_grouped_linear_gather",
+    "moe_grouped_linear_combine", "quantize_rows_dispatch",
     "moe_grouped_linear_blockscaled",
     "quantized_linear", "e4m3_encode_f32", "device_error", "set_gemm_tuning",
 ]
@@ -70,6 +71,25 @@ def quantize_rows_dynamic(X: torch.Tensor, out: tuple | None = None, fmt: str = 
     else:
         check(_lib.fp8q_quantize_rows_dynamic_fmt(X.data_ptr(), M, K, _fmt(fmt), Xq.data_ptr(), s.data_ptr(),
                                                   _stream(X)), "fp8q_quantize_rows_dynamic_fmt")
+    return Xq, s
+
+
+def quantize_rows_dispatch(X: torch.Tensor, token_rows: torch.Tensor, rows: int, out: tuple | None = None,
+                           fmt: str = "e4m3"):
+    """Per-token quantization of X fp16 [T,K] written to the expert-grouped
+    rows: token t's codes and scale go to rows token_rows[t, j] (int32
+    [T, topk], -1 = none) of the returned (uint8 [rows,K], fp32 [rows])."""
+    _need(X, torch.float16, "X", 2)
+    _need(token_rows, torch.int32, "token_rows", 2)
+    T, K = X.shape
+    if token_rows.shape[0] != T:
+        raise ValueError("token_rows must be [T, topk]")
+    Xq, s = out if out is not None else (
+        torch.empty((rows, K), dtype=torch.uint8, device=X.device),
+        torch.empty((rows,), dtype=torch.float32, device=X.device))
+    check(_lib.fp8q_quantize_rows_dispatch(X.data_ptr(), T, K, _fmt(fmt), token_rows.data_ptr(), token_rows.shape[1],
+                                           rows, Xq.data_ptr(), s.data_ptr(), _stream(X)),
+          "fp8q_quantize_rows_dispatch")
     return Xq, s
 
 
@@ -195,6 +215,32 @@ def moe_grouped_linear_gather(Xq_tok: torch.Tensor, s_x_tok: torch.Tensor, row_t
     check(_lib.fp8q_moe_grouped_linear_gather(Xq_tok.data_ptr(), s_x_tok.data_ptr(), T, row_token.data_ptr(),
                                               offsets.data_ptr(), E, rows, Wq.data_ptr(), s_w.data_ptr(), N, K,
                                               Y.data_ptr(), _stream(Xq_tok)), "fp8q_moe_grouped_linear_gather")
+    return Y
+
+
+def moe_grouped_linear_combine(Xq: torch.Tensor, s_x: torch.Tensor, offsets: torch.Tensor, Wq: torch.Tensor,
+                               s_w: torch.Tensor, row_token: torch.Tensor, row_weight: torch.Tensor, tokens: int,
+                               out: torch.Tensor | None = None) -> torch.Tensor:
+    """Expert-grouped FP8 linear whose row r is weighted by row_weight[r] and
+    added (fp16) into row row_token[r] of the [tokens, N] output (the MoE
+    down projection with the top-k combine)."""
+    _need(Xq, torch.uint8, "Xq", 2)
+    _need(s_x, torch.float32, "s_x", 1)
+    _need(offsets, torch.int32, "offsets", 1)
+    _need(Wq, torch.uint8, "Wq", 3)
+    _need(s_w, torch.float32, "s_w", 2)
+    _need(row_token, torch.int32, "row_token", 1)
+    _need(row_weight, torch.float32, "row_weight", 1)
+    rows, K = Xq.shape
+    E, N, K2 = Wq.shape
+    if (K2 != K or offsets.shape[0] != E + 1 or tuple(s_w.shape) != (E, N) or s_x.shape[0] != rows
+            or row_token.shape[0] != rows or row_weight.shape[0] != rows):
+        raise ValueError("shape mismatch")
+    Y = out if out is not None else torch.empty((tokens, N), dtype=torch.float16, device=Xq.device)
+    check(_lib.fp8q_moe_grouped_linear_combine(Xq.data_ptr(), s_x.data_ptr(), offsets.data_ptr(), E, rows,
+                                               Wq.data_ptr(), s_w.data_ptr(), N, K, row_token.data_ptr(),
+                                               row_weight.data_ptr(), tokens, Y.data_ptr(), _stream(Xq)),
+          "fp8q_moe_grouped_linear_combine")
     return Y
 
 

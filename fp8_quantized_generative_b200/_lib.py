@@ -58,6 +58,8 @@ SIGNATURES = {
     "fp8q_linear_fmt": (_INT, [_P, _INT, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "fp8q_moe_grouped_linear_fmt": (_INT, [_P, _INT, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_quantize_weight_blockwise": (_INT, [_P, _I32, _I64, _I64, _P, _P, _P]),
+    "fp8q_quantize_rows_dispatch": (_INT, [_P, _I64, _I64, _I32, _P, _I32, _I64, _P, _P, _P]),
+    "fp8q_moe_grouped_linear_combine": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P, _I64, _P, _P]),
     "fp8q_moe_grouped_linear_gather": (_INT, [_P, _P, _I64, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_moe_grouped_linear_blockscaled": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_e4m3_encode_f32": (_INT, [_P, _I64, _P, _P]),
@@ -146,6 +148,16 @@ def fp8q_moe_grouped_linear_fmt(Xq, x_fmt, s_x, offsets, E, rows, Wq, s_w, N, K,
 def fp8q_moe_grouped_linear_gather(Xq_tok, s_x_tok, tokens, row_token, offsets, E, rows, Wq, s_w, N, K, Y, stream):
     return lib().fp8q_moe_grouped_linear_gather(Xq_tok, s_x_tok, tokens, row_token, offsets, E, rows, Wq, s_w, N, K,
                                                 Y, stream)
+
+
+def fp8q_quantize_rows_dispatch(X, T, K, fmt, token_rows, topk, rows, Xq, s_x, stream):
+    return lib().fp8q_quantize_rows_dispatch(X, T, K, fmt, token_rows, topk, rows, Xq, s_x, stream)
+
+
+def fp8q_moe_grouped_linear_combine(Xq, s_x, offsets, E, rows, Wq, s_w, N, K, row_token, row_weight, tokens, out,
+                                    stream):
+    return lib().fp8q_moe_grouped_linear_combine(Xq, s_x, offsets, E, rows, Wq, s_w, N, K, row_token, row_weight,
+                                                 tokens, out, stream)
 
 
 def fp8q_quantize_weight_blockwise(W, E, N, K, Wq, s_wb, stream):

@@ -238,8 +238,8 @@ fp8q_status launch_gemm(const uint8_t* A, int64_t a_rows, const uint8_t* B, int6
   if (s != FP8Q_OK) return s;
   s = make_operand_map(&tb, B, b_rows, p.K, BN);
   if (s != FP8Q_OK) return s;
-  CUtensorMap ty;
-  s = make_output_map(&ty, p.Y, p.rows, p.N);
+  CUtensorMap ty;   // combine: Y is the [tokens, N] output, written by atomic adds only
+  s = make_output_map(&ty, p.Y, p.comb_token != nullptr ? p.tokens : p.rows, p.N);
   if (s != FP8Q_OK) return s;
   auto kernel = fp8_gemm_kernel<BN, STAGES, kGrouped, kGather>;
   const size_t smem = L::smem_bytes(kGrouped ? p.E : 0);
@@ -659,6 +659,31 @@ fp8q_status fp8q_quantize_rows_dynamic_fmt(const void* X_f16, int64_t M, int64_t
   return quantize(X_f16, M, K, Xq, s_x, stream, fmt);
 }
 
+fp8q_status fp8q_quantize_rows_dispatch(const void* X_f16, int64_t T, int64_t K, fp8q_format fmt,
+                                        const int32_t* token_rows, int32_t topk, int64_t rows, uint8_t* Xq,
+                                        float* s_x, void* stream) {
+  if (!valid_fmt(fmt)) return invalid("fmt must be FP8Q_FMT_E4M3 or FP8Q_FMT_E5M2");
+  if (topk < 1 || topk > 8) return invalid("topk must be in [1, 8]");
+  if (rows < 0 || rows > kMaxDim || rows * K > (int64_t(1) << 40)) return invalid("rows out of range");
+  fp8q_status s = check_quant_args(X_f16, T, K, rows > 0 ? Xq : nullptr, rows > 0 ? s_x : nullptr);
+  if (s != FP8Q_OK) return s;
+  if (T == 0) return FP8Q_OK;
+  if (rows == 0) return invalid("tokens with no grouped rows");
+  if (token_rows == nullptr || (reinterpret_cast<uintptr_t>(token_rows) & 3u) != 0)
+    return invalid("token_rows pointer");
+  RowDispatch d;
+  d.rows = token_rows;
+  d.topk = topk;
+  d.out_rows = static_cast<int>(rows);
+  const __half* Xh = static_cast<const __half*>(X_f16);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = fmt == FP8Q_FMT_E5M2
+                            ? launch_quant_rows<kFmtE5M2>(Xh, static_cast<int>(T), static_cast<int>(K), Xq, s_x, st, d)
+                            : launch_quant_rows<kFmtE4M3>(Xh, static_cast<int>(T), static_cast<int>(K), Xq, s_x, st, d);
+  if (e != cudaSuccess) return cuda_fail(e, "quant_rows dispatch launch");
+  return FP8Q_OK;
+}
+
 fp8q_status fp8q_quantize_weight_per_tensor(const void* W_f16, int64_t N, int64_t K, uint8_t* Wq, float* s_w,
                                             void* stream) {
   if (N == 0) return invalid("N must be positive");
@@ -829,6 +854,47 @@ fp8q_status fp8q_moe_grouped_linear_gather(const uint8_t* Xq_tok, const float* s
   const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBNGrouped - 1) / kBNGrouped);
   // the A tensor map (token matrix) is built but unused: the producer gathers the rows
   return launch_gemm<true, true>(Xq_tok, tokens, Wq, int64_t(E) * N, p, tiles, static_cast<cudaStream_t>(stream));
+}
+
+fp8q_status fp8q_moe_grouped_linear_combine(const uint8_t* Xq, const float* s_x, const int32_t* offsets, int32_t E,
+                                            int64_t rows, const uint8_t* Wq, const float* s_w, int64_t N, int64_t K,
+                                            const int32_t* row_token, const float* row_weight, int64_t tokens,
+                                            void* out_f16, void* stream) {
+  if (E < 1 || E > kMaxExperts) return invalid("E must be in [1, 1024]");
+  if (rows < 0 || rows > kMaxDim) return invalid("rows out of range");
+  if (tokens <= 0 || tokens > kMaxDim || tokens * N > (int64_t(1) << 40)) return invalid("tokens out of range");
+  if (N <= 0 || N % 8 != 0 || int64_t(E) * N > kMaxDim) return invalid("N must be positive, a multiple of 8, E*N < 2^31");
+  if (K <= 0 || K > kMaxDim || K % 16 != 0) return invalid("K must be positive and a multiple of 16");
+  if (offsets == nullptr || (reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return invalid("offsets pointer");
+  if (rows > 0 && (row_token == nullptr || (reinterpret_cast<uintptr_t>(row_token) & 3u) != 0))
+    return invalid("row_token pointer");
+  if (rows > 0 && (row_weight == nullptr || (reinterpret_cast<uintptr_t>(row_weight) & 3u) != 0))
+    return invalid("row_weight pointer");
+  if (!aligned16(out_f16)) return invalid("null or non-16-byte-aligned output");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(out_f16, 0, static_cast<size_t>(tokens * N) * sizeof(__half), st);
+  if (e != cudaSuccess) return cuda_fail(e, "combine output clear");
+  if (rows == 0) return FP8Q_OK;   // every row-side pointer may be null
+  if (!aligned16(Xq) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_w))
+    return invalid("null or non-16-byte-aligned pointer");
+  GemmParams p = {};   // every field set below; zero for the rest
+  p.s_x = s_x;
+  p.s_w = s_w;
+  p.Y = static_cast<__half*>(out_f16);
+  p.offsets = offsets;
+  p.rows = static_cast<int>(rows);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.E = E;
+  p.tail_q = 1;
+  p.l2_prefetch = l2_prefetch_enabled();
+  p.half_tiles = knobs().half_tiles;
+  p.x_fmt = FP8Q_FMT_E4M3;
+  p.tokens = static_cast<int>(tokens);
+  p.comb_token = row_token;
+  p.comb_weight = row_weight;
+  const int64_t tiles = ((rows + kBM - 1) / kBM + E) * ((N + kBNGrouped - 1) / kBNGrouped);
+  return launch_gemm<true>(Xq, rows, Wq, int64_t(E) * N, p, tiles, st);
 }
 
 fp8q_status fp8q_quantize_weight_blockwise(const void* W_f16, int32_t E, int64_t N, int64_t K, uint8_t* Wq,

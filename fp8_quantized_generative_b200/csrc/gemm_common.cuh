@@ -47,7 +47,9 @@ struct GemmParams {
   int x_fmt;                // activation code format (Fp8Fmt): E4M3, or E5M2 for the variant
   const uint8_t* xq;        // grouped gather: the token matrix of activation codes [tokens, K]
   const int32_t* row_token; // grouped gather: row r of the product reads token row_token[r] (nullptr: row r)
-  int tokens;               // grouped gather: rows of the token matrix
+  int tokens;               // grouped gather / combine: rows of the token matrix
+  const int32_t* comb_token; // combine: grouped row r adds into output row comb_token[r] (nullptr: plain store)
+  const float* comb_weight;  // combine: the weight of grouped row r
 };
 
 // Row of the activation codes / scales that product row r reads (the row
@@ -117,6 +119,8 @@ template <int kMaxChunks>
 struct EpiScales {
   float sx;
   float sw[kMaxChunks];
+  float rw;    // combine: weight of this lane's row
+  int ctok;    // combine: output (token) row of this lane's row, -1: none
 };
 
 template <int kMaxChunks>
@@ -125,6 +129,17 @@ __device__ __forceinline__ EpiScales<kMaxChunks> epilogue_scales(const EpiTile& 
   EpiScales<kMaxChunks> e;
   const int r = w.qrow0 + lane;
   e.sx = r < t.row_end ? __ldg(p.s_x + act_row(p, r)) : 0.0f;
+  e.rw = 0.0f;
+  e.ctok = -1;
+  if (p.comb_token != nullptr && r < t.row_end) {
+    const int tk = __ldg(p.comb_token + r);
+    if (tk >= 0 && tk < p.tokens) {
+      e.ctok = tk;
+      e.rw = __ldg(p.comb_weight + r);
+    } else {
+      raise_error(0x8u);
+    }
+  }
 #pragma unroll
   for (int j = 0; j < kMaxChunks; ++j) {
     const int cl = w.col0 + j * 32 + lane;
@@ -156,7 +171,12 @@ __device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams
   const int qrow0 = w.qrow0;
   const int valid = t.row_end - qrow0;   // rows of this warp that are stored (<= 0: none)
   if (valid <= 0) return;
-  const bool bulk = t.clip || valid >= 32;
+  // MoE combine: rows go back to their tokens with fp16 atomic adds, read
+  // from the staging tile four lanes to a row so that each instruction adds
+  // whole 32-byte sectors (half as many L2 atomic operations as one lane per
+  // row, 16 bytes at a time).
+  const bool combine = p.comb_token != nullptr;
+  const bool bulk = !combine && (t.clip || valid >= 32);
   const uint32_t taddr0 = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(w.tcol0);
   uint32_t v[2][32];
   tmem_ld_32x32b_x32(taddr0, v[0]);
@@ -175,8 +195,12 @@ __device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams
     for (int i = 0; i < 16; ++i) {
       const float w0 = __shfl_sync(0xffffffffu, pre.sw[j], 2 * i);
       const float w1 = __shfl_sync(0xffffffffu, pre.sw[j], 2 * i + 1);
-      const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i]), pre.sx), w0);
-      const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i + 1]), pre.sx), w1);
+      float y0 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i]), pre.sx), w0);
+      float y1 = __fmul_rn(__fmul_rn(__uint_as_float(cur[2 * i + 1]), pre.sx), w1);
+      if (combine) {
+        y0 = __fmul_rn(y0, pre.rw);
+        y1 = __fmul_rn(y1, pre.rw);
+      }
       const __half2 hv = __floats2half2_rn(y0, y1);
       packed[i] = *reinterpret_cast<const uint32_t*>(&hv);
     }
@@ -207,8 +231,12 @@ __device__ __forceinline__ void epilogue_slab(const EpiTile& t, const GemmParams
         const int c = lane & 3;
         const uint4 val = ld_shared_v4(sbase + stage_off(rr, c));
         const int gcol = t.n0 + cl + c * 8;
-        if (rr < valid && gcol < p.N)
+        if (combine) {
+          const int tok = __shfl_sync(0xffffffffu, pre.ctok, rr);   // -1: past the group or rejected
+          if (tok >= 0 && gcol < p.N) red_add_f16x8(p.Y + static_cast<int64_t>(tok) * p.N + gcol, val.x, val.y, val.z, val.w);
+        } else if (rr < valid && gcol < p.N) {
           *reinterpret_cast<uint4*>(p.Y + static_cast<int64_t>(qrow0 + rr) * p.N + gcol) = val;
+        }
       }
       __syncwarp();
     }

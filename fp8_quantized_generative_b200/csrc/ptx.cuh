@@ -325,6 +325,14 @@ __device__ __forceinline__ void mma_commit_pair_mc(uint64_t* bar, uint16_t cta_m
       : "memory");
 }
 
+// ---------------------------------------------------------------- FP16 scatter-add (MoE combine)
+// out[0..7] += the eight fp16 values packed in v (one 16-byte vector atomic add,
+// each element rounded to nearest even); addr 16-byte aligned.
+__device__ __forceinline__ void red_add_f16x8(__half* addr, uint32_t v0, uint32_t v1, uint32_t v2, uint32_t v3) {
+  asm volatile("red.global.add.noftz.v4.f16x2 [%0], {%1, %2, %3, %4};" ::"l"(addr), "r"(v0), "r"(v1), "r"(v2), "r"(v3)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async (row gathers)
 // 16-byte global -> shared copy; src_bytes < 16 zero-fills the rest (0: all zero, src not read).
 __device__ __forceinline__ void cp_async_16_zfill(uint32_t smem_dst, const void* src, uint32_t src_bytes) {

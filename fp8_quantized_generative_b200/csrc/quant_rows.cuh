@@ -66,12 +66,48 @@ __device__ __forceinline__ uint2 encode8(const uint4& v, float r) {
   return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
+// Output rows of the quantizer.  Plain: input row m writes output row m.
+// Dispatch (MoE, a token feeding top-k experts): input row m writes output
+// rows rows[m * topk + j] for j < topk, the token's rows in the expert-grouped
+// matrix (-1: none), so each token is read and encoded once.  An entry
+// outside [-1, out_rows) sets error bit 0x8 and is skipped.
+struct RowDispatch {
+  const int32_t* rows = nullptr;
+  int topk = 0;
+  int out_rows = 0;
+};
+
+template <int VPT>
+__device__ __forceinline__ void store_row_codes(const RowDispatch& d, int row, int t, int tpr, int nvec, int K,
+                                                const uint2 (&enc)[VPT], float s, uint8_t* __restrict__ Q,
+                                                float* __restrict__ S) {
+  const int n = d.rows == nullptr ? 1 : d.topk;
+  for (int k = 0; k < n; ++k) {
+    int orow = row;
+    if (d.rows != nullptr) {
+      orow = __ldg(d.rows + static_cast<int64_t>(row) * d.topk + k);
+      if (orow < 0 || orow >= d.out_rows) {
+        if (orow != -1 && t == 0) raise_error(0x8u);
+        continue;
+      }
+    }
+    uint2* dst = reinterpret_cast<uint2*>(Q + static_cast<int64_t>(orow) * K);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int j = t + i * tpr;
+      if (j < nvec) dst[j] = enc[i];
+    }
+    if (t == 0) S[orow] = s;
+  }
+}
+
 // Grid: ceil(M / (CTA / TPR)) CTAs of CTA threads; TPR threads per row.
 // With few rows, small CTAs (two rows of one warp each) spread them over more
 // SMs: the grid is a single wave, so its time is that of the most loaded SM.
 template <int TPR, int VPT, int F, int CTA = 256>
 __global__ void __launch_bounds__(CTA) quant_rows_kernel(const __half* __restrict__ X, int M, int K,
-                                                        uint8_t* __restrict__ Q, float* __restrict__ S) {
+                                                        uint8_t* __restrict__ Q, float* __restrict__ S,
+                                                        const RowDispatch d) {
   static_assert(TPR >= 32 && TPR <= CTA && CTA <= 256 && (TPR & (TPR - 1)) == 0, "TPR");
   // Programmatic dependent launch: let the next kernel start its set-up now
   // (it waits for this grid before touching our outputs), and wait for the
@@ -114,19 +150,17 @@ __global__ void __launch_bounds__(CTA) quant_rows_kernel(const __half* __restric
   if (!live) return;
 
   const RowScale rs = row_scale_from_amax<F>(m);
-  uint2* dst = reinterpret_cast<uint2*>(Q + static_cast<int64_t>(row) * K);
+  uint2 enc[VPT];
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int j = t + i * TPR;
-    if (j < nvec) dst[j] = encode8<F>(v[i], rs.r);
-  }
-  if (t == 0) S[row] = rs.s;
+  for (int i = 0; i < VPT; ++i) enc[i] = encode8<F>(v[i], rs.r);
+  store_row_codes<VPT>(d, row, t, TPR, nvec, K, enc, rs.s, Q, S);
 }
 
 // Any K (multiple of 8): one CTA of 256 threads per row, two passes over the row.
 template <int F>
 __global__ void __launch_bounds__(256) quant_rows_long_kernel(const __half* __restrict__ X, int M, int K,
-                                                             uint8_t* __restrict__ Q, float* __restrict__ S) {
+                                                             uint8_t* __restrict__ Q, float* __restrict__ S,
+                                                             const RowDispatch d) {
   __shared__ float red[8];
   pdl_launch_dependents();
   pdl_wait_prior_grid();
@@ -142,9 +176,20 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const __half* __re
 #pragma unroll
   for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
   const RowScale rs = row_scale_from_amax<F>(m);
-  uint2* dst = reinterpret_cast<uint2*>(Q + static_cast<int64_t>(row) * K);
-  for (int j = threadIdx.x; j < nvec; j += 256) dst[j] = encode8<F>(__ldg(src + j), rs.r);
-  if (threadIdx.x == 0) S[row] = rs.s;
+  const int n = d.rows == nullptr ? 1 : d.topk;
+  for (int k = 0; k < n; ++k) {   // (re-encoded per output row: the row does not fit in registers)
+    int orow = row;
+    if (d.rows != nullptr) {
+      orow = __ldg(d.rows + static_cast<int64_t>(row) * d.topk + k);
+      if (orow < 0 || orow >= d.out_rows) {
+        if (orow != -1 && threadIdx.x == 0) raise_error(0x8u);
+        continue;
+      }
+    }
+    uint2* dst = reinterpret_cast<uint2*>(Q + static_cast<int64_t>(orow) * K);
+    for (int j = threadIdx.x; j < nvec; j += 256) dst[j] = encode8<F>(__ldg(src + j), rs.r);
+    if (threadIdx.x == 0) S[orow] = rs.s;
+  }
 }
 
 // ------------------------------------------------------------ per-tensor (E4M3)
@@ -235,12 +280,13 @@ inline cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cu
 
 // Host-side launcher: picks (TPR, VPT) so one row fits in registers.
 template <int F = kFmtE4M3>
-inline cudaError_t launch_quant_rows(const __half* X, int M, int K, uint8_t* Q, float* S, cudaStream_t st) {
+inline cudaError_t launch_quant_rows(const __half* X, int M, int K, uint8_t* Q, float* S, cudaStream_t st,
+                                     const RowDispatch d = RowDispatch{}) {
   const int nvec = K / 8;
   int tpr = 32;
   while (tpr < 256 && tpr * 8 < nvec) tpr *= 2;
   const int vpt_needed = (nvec + tpr - 1) / tpr;
-  if (vpt_needed > 8) return launch_pdl(quant_rows_long_kernel<F>, dim3(M), dim3(256), st, X, M, K, Q, S);
+  if (vpt_needed > 8) return launch_pdl(quant_rows_long_kernel<F>, dim3(M), dim3(256), st, X, M, K, Q, S, d);
   const int vpt = vpt_needed <= 1 ? 1 : vpt_needed <= 2 ? 2 : vpt_needed <= 4 ? 4 : 8;
   // Few rows (fewer than 256 CTAs of 256 threads, i.e. under ~2 per SM):
   // CTAs of 64 threads spread them over more SMs (measured 10% faster at
@@ -252,8 +298,8 @@ inline cudaError_t launch_quant_rows(const __half* X, int M, int K, uint8_t* Q, 
   const dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
 #define FP8Q_QR_CASE(T, V)                                                                                      \
   if (tpr == T && vpt == V)                                                                                   \
-    return small ? launch_pdl(quant_rows_kernel<T, V, F, (T < 64 ? 64 : T)>, grid, dim3(cta), st, X, M, K, Q, S) \
-                 : launch_pdl(quant_rows_kernel<T, V, F, 256>, grid, dim3(cta), st, X, M, K, Q, S);
+    return small ? launch_pdl(quant_rows_kernel<T, V, F, (T < 64 ? 64 : T)>, grid, dim3(cta), st, X, M, K, Q, S, d) \
+                 : launch_pdl(quant_rows_kernel<T, V, F, 256>, grid, dim3(cta), st, X, M, K, Q, S, d);
   FP8Q_QR_CASE(32, 1) FP8Q_QR_CASE(32, 2) FP8Q_QR_CASE(32, 4) FP8Q_QR_CASE(32, 8)
   FP8Q_QR_CASE(64, 8) FP8Q_QR_CASE(128, 8) FP8Q_QR_CASE(256, 8)
 #undef FP8Q_QR_CASE

@@ -158,6 +158,19 @@ def gate_weights(logits_f16: np.ndarray, experts: np.ndarray) -> np.ndarray:
     return (z / z.sum(axis=1, keepdims=True)).astype(np.float32)
 
 
+def token_rows(row_token: np.ndarray, tokens: int, topk: int = MOE_TOPK) -> np.ndarray:
+    """Inverse of the grouping: int32 [tokens, topk], the grouped rows of each
+    token in row order (-1 where a token has fewer than topk rows)."""
+    out = np.full((tokens, topk), -1, dtype=np.int32)
+    fill = np.zeros(tokens, dtype=np.int64)
+    for r, t in enumerate(np.asarray(row_token, dtype=np.int64)):
+        if fill[t] >= topk:
+            raise ValueError(f"token {t} has more than {topk} rows")
+        out[t, fill[t]] = r
+        fill[t] += 1
+    return out
+
+
 def row_weights(weights: np.ndarray, experts: np.ndarray) -> np.ndarray:
     """The combine weight of every grouped row (same order as group_by_expert): float32 [T*topk]."""
     return weights.reshape(-1)[_expert_order(experts)].astype(np.float32)

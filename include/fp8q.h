@@ -261,6 +261,39 @@ fp8q_status fp8q_moe_grouped_linear_gather(const uint8_t* Xq_tok, const float* s
                                            int64_t rows, const uint8_t* Wq, const float* s_w,
                                            int64_t N, int64_t K, void* Y_f16, void* stream);
 
+/*
+ * MoE expert grouped linear with the top-k combine in its epilogue (the down
+ * projection of the MoE layer) [P1 关键证据 item 2; P2 §3.2]: grouped row r
+ * (inputs and offsets as for fp8q_moe_grouped_linear) produces
+ * y = (acc * s_x[r]) * s_w[e, n] in fp32 and adds fp16(y * row_weight[r])
+ * into row row_token[r] of out_f16 [tokens, N] with an fp16 atomic add
+ * (round to nearest).  The call first zeroes out_f16 (cudaMemsetAsync on
+ * `stream`).  With at most two rows per token the result does not depend on
+ * the order of the additions.  row_token int32 [rows], row_weight fp32
+ * [rows] (the router's combine weights), device.  A row_token entry outside
+ * [0, tokens) sets FP8Q_DEVERR_BAD_OFFSETS and that row adds nothing.
+ */
+fp8q_status fp8q_moe_grouped_linear_combine(const uint8_t* Xq, const float* s_x,
+                                            const int32_t* offsets, int32_t E, int64_t rows,
+                                            const uint8_t* Wq, const float* s_w, int64_t N, int64_t K,
+                                            const int32_t* row_token, const float* row_weight,
+                                            int64_t tokens, void* out_f16, void* stream);
+
+/*
+ * Per-token activation quantization with the MoE dispatch in its store
+ * [P2 §2.2 per-token activation scales; §3.2 tokens grouped by expert]:
+ * token row t of X_f16 [T, K] is quantized once (the steps of
+ * fp8q_quantize_rows_dynamic_fmt, format fmt) and its codes and scale are
+ * written to every grouped row token_rows[t * topk + j], j < topk, of Xq
+ * [rows, K] and s_x [rows] -- the expert-grouped activation matrix the MoE
+ * grouped linear reads.  token_rows int32 [T, topk], device; -1 = no row.
+ * A grouped row no entry names is left unwritten.  An entry outside
+ * [-1, rows) sets FP8Q_DEVERR_BAD_OFFSETS and is skipped.  topk in [1, 8].
+ */
+fp8q_status fp8q_quantize_rows_dispatch(const void* X_f16, int64_t T, int64_t K, fp8q_format fmt,
+                                        const int32_t* token_rows, int32_t topk, int64_t rows, uint8_t* Xq,
+                                        float* s_x, void* stream);
+
 /* fp8q_moe_grouped_linear with the activation codes Xq in format x_fmt. */
 fp8q_status fp8q_moe_grouped_linear_fmt(const uint8_t* Xq, fp8q_format x_fmt, const float* s_x,
                                         const int32_t* offsets, int32_t E, int64_t rows,

@@ -170,3 +170,32 @@ def test_gather_rejects(L):
     assert g(a, a, 10, a, a, 4, 8, a, a, 12, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
     assert g(BAD, a, 10, a, a, 4, 8, a, a, 16, 32, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
     assert g(0, 0, 10, a, a, 4, 0, 0, 0, 16, 32, 0, 0) == _lib.FP8Q_OK                  # no rows
+
+
+def test_combine_rejects(L):
+    a = 0x1000
+    c = _lib.fp8q_moe_grouped_linear_combine
+    #      Xq s_x off E  rows Wq s_w N   K  tok w  T   out st
+    assert c(a, a, a, 4, 8, a, a, 16, 32, a, a, 0, a, 0) == _lib.FP8Q_ERR_INVALID_ARG     # no tokens
+    assert c(a, a, a, 0, 8, a, a, 16, 32, a, a, 4, a, 0) == _lib.FP8Q_ERR_INVALID_ARG     # E = 0
+    assert c(a, a, a, 4, 8, a, a, 12, 32, a, a, 4, a, 0) == _lib.FP8Q_ERR_INVALID_ARG     # N % 8
+    assert c(a, a, a, 4, 8, a, a, 16, 24, a, a, 4, a, 0) == _lib.FP8Q_ERR_INVALID_ARG     # K % 16
+    assert c(a, a, a, 4, 8, a, a, 16, 32, 0, a, 4, a, 0) == _lib.FP8Q_ERR_INVALID_ARG     # null row_token
+    assert c(a, a, a, 4, 8, a, a, 16, 32, a, 0x1002, 4, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert c(a, a, a, 4, 8, a, a, 16, 32, a, a, 4, BAD, 0) == _lib.FP8Q_ERR_INVALID_ARG   # output alignment
+    assert c(a, a, 0x1002, 4, 8, a, a, 16, 32, a, a, 4, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+
+
+def test_dispatch_rejects(L):
+    a = 0x1000
+    d = _lib.fp8q_quantize_rows_dispatch
+    #      X  T   K   fmt tr topk rows Xq s  st
+    assert d(a, 4, 32, 0, a, 0, 8, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG      # topk 0
+    assert d(a, 4, 32, 0, a, 9, 8, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG      # topk > 8
+    assert d(a, 4, 32, 2, a, 2, 8, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG      # fmt
+    assert d(a, 4, 24, 0, a, 2, 8, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG      # K % 16
+    assert d(a, 4, 32, 0, 0, 2, 8, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG      # null token_rows
+    assert d(a, 4, 32, 0, 0x1002, 2, 8, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert d(a, 4, 32, 0, a, 2, 8, BAD, a, 0) == _lib.FP8Q_ERR_INVALID_ARG    # Xq alignment
+    assert d(a, 4, 32, 0, a, 2, 0, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG      # tokens, no rows
+    assert d(0, 0, 32, 0, 0, 2, 0, 0, 0, 0) == _lib.FP8Q_OK                   # nothing to do

@@ -1,0 +1,195 @@
+"""GPU parity of the MoE down projection with the top-2 combine in its
+epilogue (fp8q_moe_grouped_linear_combine; 'FP8量化在生成式推荐系统OneRec-V2中的
+优化实践' §3.2 and the OneRec-V2 item on per-token/expert-aligned quantization
+of the MoE layer): grouped row r adds fp16(row_weight[r] * y[r]) into output
+row row_token[r] with an FP16 atomic add.
+
+Tolerance.  out[t] = c1 + c2 can cancel, so an error bound relative to
+|out[t]| is wrong; each contribution carries the grouped linear's error
+(2^-9 |c| + 1e-3 rms) and the sum one more fp16 rounding on either side, so
+the bound is taken against S[t] = sum_r |row_weight[r] * y[r]|:
+    per element:  |out_gpu - out_ref| <= 2^-9 * (S + |out_ref|) + 1e-3 * rms(S)
+    whole tensor: ||out_gpu - out_ref||_F <= 1e-3 * ||S||_F
+Kernel-against-kernel checks are bitwise: with unit weights the combine
+equals the fp16 scatter-add (one rounding of the exact sum) of the plain
+grouped linear's outputs, since the same tiles produce the same fp32 values.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_combine_ref, moe_ref, quant_rows
+from fp8_quantized_generative_b200 import workloads as wl
+
+from parity import assert_no_device_error, sample_rows, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fq():
+    import fp8_quantized_generative_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def routed(T, E, seed, topk=2):
+    logits = wl.random_f16((T, E), seed=seed).numpy()
+    experts = wl.route_top2(logits, topk=topk)
+    row_token, offsets = wl.group_by_expert(experts, E)
+    w = wl.row_weights(wl.gate_weights(logits, experts), experts)
+    return row_token.astype(np.int32), np.asarray(offsets, dtype=np.int32), w.astype(np.float32)
+
+
+def oracle_quant(X, W):
+    E, N, K = W.shape
+    xq, sx = quant_rows(X.numpy())
+    q = [quant_rows(W[e].numpy()) for e in range(E)]
+    return xq, sx, np.stack([c for c, _ in q]), np.stack([s for _, s in q])
+
+
+def assert_close_combine(got, ref, S, what):
+    g = np.asarray(got, np.float64)
+    r = np.asarray(ref, np.float64)
+    assert g.shape == r.shape and np.all(np.isfinite(g)), what
+    rms = float(np.sqrt(np.mean(S * S)))
+    bound = 2.0 ** -9 * (S + np.abs(r)) + 1e-3 * rms
+    bad = np.abs(g - r) > bound
+    if np.any(bad):
+        i = tuple(np.argwhere(bad)[0])
+        raise AssertionError(f"{what}: {int(bad.sum())} out of tolerance; first at {i}: gpu={g[i]!r} "
+                             f"ref={r[i]!r} bound={bound[i]!r}")
+    assert np.linalg.norm(g - r) <= 1e-3 * np.linalg.norm(S), what
+
+
+def magnitude_sum(xq, sx, offsets, wq, sw, row_token, w, T):
+    """S[t] = sum over t's rows of |w_r * y_r| (y from the oracle's grouped linear)."""
+    y = moe_ref(xq, sx, offsets, wq, sw).astype(np.float64)
+    S = np.zeros((T, y.shape[1]))
+    np.add.at(S, row_token.astype(np.int64), np.abs(w.astype(np.float64))[:, None] * np.abs(y))
+    return S
+
+
+def run_combine(fq, Xp, offsets, W, row_token, w, T):
+    Xq, s_x = fq.quantize_rows_dynamic(Xp.cuda())
+    Wq, s_w = fq.quantize_weight_per_channel(W.cuda())
+    out = torch.full((T, W.shape[1]), float("nan"), dtype=torch.float16, device="cuda")
+    fq.moe_grouped_linear_combine(Xq, s_x, torch.from_numpy(offsets).cuda(), Wq, s_w,
+                                  torch.from_numpy(row_token).cuda(), torch.from_numpy(w).cuda(), T, out=out)
+    torch.cuda.synchronize()
+    return out, (Xq, s_x, Wq, s_w)
+
+
+@pytest.mark.parametrize("T,E,N,K", [(40, 6, 264, 272), (300, 8, 256, 512), (1, 3, 64, 128), (700, 5, 136, 1040)])
+def test_routed_top2_against_oracle(fq, T, E, N, K):
+    row_token, offsets, w = routed(T, E, seed=T + 7 * E)
+    Xp = wl.random_f16((len(row_token), K), seed=T + K)
+    W = wl.random_f16((E, N, K), seed=E + N, std=0.02)
+    out, _ = run_combine(fq, Xp, offsets, W, row_token, w, T)
+    xq, sx, wq, sw = oracle_quant(Xp, W)
+    ref = moe_combine_ref(xq, sx, offsets, wq, sw, row_token, w, T)
+    S = magnitude_sum(xq, sx, offsets, wq, sw, row_token, w, T)
+    assert_close_combine(to_np(out), ref, S, f"combine T={T} E={E} N={N} K={K}")
+    assert_no_device_error()
+
+
+def test_tokens_without_rows_are_zero(fq):
+    T, E, N, K = 50, 3, 128, 256
+    row_token = np.array([0, 3, 3, 7, 0, 9], np.int32)        # tokens 1,2,4,5,6,8,10.. get nothing
+    offsets = np.array([0, 2, 2, 6], np.int32)
+    w = np.array([0.25, 0.5, 0.5, 1.0, 0.75, -0.5], np.float32)
+    Xp = wl.random_f16((6, K), seed=5)
+    W = wl.random_f16((E, N, K), seed=6, std=0.02)
+    out, _ = run_combine(fq, Xp, offsets, W, row_token, w, T)
+    xq, sx, wq, sw = oracle_quant(Xp, W)
+    ref = moe_combine_ref(xq, sx, offsets, wq, sw, row_token, w, T)
+    S = magnitude_sum(xq, sx, offsets, wq, sw, row_token, w, T)
+    assert_close_combine(to_np(out), ref, S, "sparse tokens")
+    untouched = np.setdiff1d(np.arange(T), row_token)
+    assert np.all(to_np(out)[untouched].view(np.uint16) == 0)        # +0.0 exactly
+    assert_no_device_error()
+
+
+def test_no_rows_clears_output(fq):
+    T, E, N, K = 9, 2, 64, 128
+    out = torch.full((T, N), 3.0, dtype=torch.float16, device="cuda")
+    Xq = torch.empty((0, K), dtype=torch.uint8, device="cuda")
+    s_x = torch.empty((0,), dtype=torch.float32, device="cuda")
+    Wq, s_w = fq.quantize_weight_per_channel(wl.random_f16((E, N, K), seed=1, std=0.02).cuda())
+    off = torch.zeros(E + 1, dtype=torch.int32, device="cuda")
+    e32 = torch.empty((0,), dtype=torch.int32, device="cuda")
+    ef = torch.empty((0,), dtype=torch.float32, device="cuda")
+    fq.moe_grouped_linear_combine(Xq, s_x, off, Wq, s_w, e32, ef, T, out=out)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+
+
+@pytest.mark.parametrize("topk", [1, 2])
+def test_unit_weights_equal_scatter_add_of_grouped_linear(fq, topk):
+    T, E, N, K = 400, 7, 512, 768
+    row_token, offsets, _ = routed(T, E, seed=21 + topk, topk=topk)
+    ones = np.ones(len(row_token), np.float32)
+    Xp = wl.random_f16((len(row_token), K), seed=22)
+    W = wl.random_f16((E, N, K), seed=23, std=0.02)
+    out, (Xq, s_x, Wq, s_w) = run_combine(fq, Xp, offsets, W, row_token, ones, T)
+    fq.set_gemm_tuning(1, 0, 0)           # the single-CTA grouped kernel, as the combine uses
+    try:
+        Y = fq.moe_grouped_linear(Xq, s_x, torch.from_numpy(offsets).cuda(), Wq, s_w)
+        torch.cuda.synchronize()
+    finally:
+        fq.set_gemm_tuning(0, 0, 0)
+    y = to_np(Y).astype(np.float64)
+    exp = np.zeros((T, N), np.float64)
+    np.add.at(exp, row_token.astype(np.int64), y)          # exact: two fp16 values sum exactly in fp64
+    exp = exp.astype(np.float16)
+    assert np.array_equal(to_np(out).view(np.uint16), exp.view(np.uint16))
+
+
+def test_repeatable_bitwise(fq):
+    T, E, N, K = 600, 8, 384, 512
+    row_token, offsets, w = routed(T, E, seed=31)
+    Xp = wl.random_f16((len(row_token), K), seed=32)
+    W = wl.random_f16((E, N, K), seed=33, std=0.02)
+    a, _ = run_combine(fq, Xp, offsets, W, row_token, w, T)
+    b, _ = run_combine(fq, Xp, offsets, W, row_token, w, T)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_bad_token_is_reported(fq):
+    T, E, N, K = 8, 2, 64, 128
+    Xq, s_x = fq.quantize_rows_dynamic(wl.random_f16((6, K), seed=3).cuda())
+    Wq, s_w = fq.quantize_weight_per_channel(wl.random_f16((E, N, K), seed=4, std=0.02).cuda())
+    row_token = torch.tensor([0, 1, 2, 8, 4, 5], dtype=torch.int32, device="cuda")      # 8 >= T
+    w = torch.ones(6, dtype=torch.float32, device="cuda")
+    offsets = torch.tensor([0, 3, 6], dtype=torch.int32, device="cuda")
+    fq.moe_grouped_linear_combine(Xq, s_x, offsets, Wq, s_w, row_token, w, T)
+    assert fq.device_error() == 0x8
+
+
+def test_moe_down_combine(fq):
+    m = wl.moe()
+    row_token = np.asarray(m.token_of_row, dtype=np.int32)
+    offsets = np.asarray(m.offsets, dtype=np.int32)
+    T = m.X.shape[0]
+    R, F = len(row_token), wl.MOE_F
+    H = wl.random_f16((R, F), seed=404)                 # the expert FFN's hidden rows
+    out, _ = run_combine(fq, H, offsets, m.W_down, row_token, m.row_weight, T)
+    # oracle on sampled tokens: both rows of each sampled token, each with its expert
+    toks = sample_rows(T, 96, seed=13)
+    pick = np.flatnonzero(np.isin(row_token, toks))
+    expert_of = np.searchsorted(offsets.astype(np.int64), pick, side="right") - 1
+    order = np.argsort(expert_of, kind="stable")
+    pick, expert_of = pick[order], expert_of[order]
+    E = m.W_down.shape[0]
+    sub_off = np.searchsorted(expert_of, np.arange(E + 1), side="left").astype(np.int64)
+    xq, sx = quant_rows(H.numpy()[pick])
+    used = np.unique(expert_of)
+    wq = np.zeros((E,) + tuple(m.W_down.shape[1:]), np.uint8)
+    sw = np.zeros(m.W_down.shape[:2], np.float32)
+    for e in used:
+        wq[e], sw[e] = quant_rows(m.W_down[e].numpy())
+    tok_local = np.searchsorted(toks, row_token[pick])
+    ref = moe_combine_ref(xq, sx, sub_off, wq, sw, tok_local, m.row_weight[pick], len(toks))
+    S = magnitude_sum(xq, sx, sub_off, wq, sw, tok_local, m.row_weight[pick], len(toks))
+    assert_close_combine(to_np(out)[toks], ref, S, "moe down combine")
+    assert_no_device_error()

@@ -101,3 +101,72 @@ def test_moe_up_from_tokens(fq):
         ref[sel] = linear_ref(xq[sel], sx[sel], wq, sw)
     assert_close_f16(to_np(Y)[rows], ref, "moe up from tokens")
     assert_no_device_error()
+
+
+# ------------------------------------------------- dispatch in the quantizer's store
+
+def run_dispatch(fq, X, token_rows, R, fmt="e4m3"):
+    Xq = torch.full((R, X.shape[1]), 0x7F, dtype=torch.uint8, device="cuda")
+    s = torch.full((R,), float("nan"), dtype=torch.float32, device="cuda")
+    fq.quantize_rows_dispatch(X.cuda(), torch.from_numpy(token_rows).cuda(), R, out=(Xq, s), fmt=fmt)
+    torch.cuda.synchronize()
+    return to_np(Xq), to_np(s)
+
+
+@pytest.mark.parametrize("T,E,K", [(40, 6, 272), (300, 8, 2048), (5, 3, 16), (9, 4, 20480)])
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_dispatch_bit_exact(fq, T, E, K, fmt):
+    # grouped row r holds the codes and scale of token row_token[r] (K = 20480: the two-pass kernel)
+    row_token, _ = routed(T, E, seed=T + K)
+    R = len(row_token)
+    X = wl.random_f16((T, K), seed=K + 1, std=2.0)
+    got_q, got_s = run_dispatch(fq, X, wl.token_rows(row_token, T), R, fmt)
+    ref_q, ref_s = quant_rows(X.numpy(), fmt)
+    assert np.array_equal(got_q, ref_q[row_token])
+    assert np.array_equal(got_s.view(np.uint32), ref_s[row_token].view(np.uint32))
+    assert_no_device_error()
+
+
+def test_dispatch_skips_minus_one_and_reports_bad_rows(fq):
+    T, K, R = 4, 128, 5
+    X = wl.random_f16((T, K), seed=2)
+    tr = np.array([[0, 3], [-1, -1], [1, -1], [4, 2]], np.int32)
+    got_q, got_s = run_dispatch(fq, X, tr, R)
+    ref_q, ref_s = quant_rows(X.numpy())
+    for t, r in [(0, 0), (0, 3), (2, 1), (3, 4), (3, 2)]:
+        assert np.array_equal(got_q[r], ref_q[t]) and got_s[r] == ref_s[t]
+    assert_no_device_error()
+    bad = np.array([[0, 5], [1, -2], [2, -1], [3, -1]], np.int32)     # 5 >= R, -2 < -1
+    got_q, _ = run_dispatch(fq, X, bad, R)
+    assert fq.device_error() == 0x8
+    assert np.array_equal(got_q[0], ref_q[0]) and np.all(got_q[4] == 0x7F)
+
+
+def test_dispatch_then_grouped_linear_equals_gather(fq):
+    # quantize once and scatter, then the plain grouped linear: bitwise the gathered product
+    T, E, N, K = 500, 10, 512, 1024
+    row_token, offsets = routed(T, E, seed=9)
+    X = wl.random_f16((T, K), seed=10)
+    W = wl.random_f16((E, N, K), seed=11, std=0.02)
+    Y, (_, _, Wq, s_w) = run_gather(fq, X, row_token, offsets, W)
+    Xq_g, s_g = fq.quantize_rows_dispatch(X.cuda(), torch.from_numpy(wl.token_rows(row_token, T)).cuda(),
+                                          len(row_token))
+    fq.set_gemm_tuning(1, 0, 0)
+    try:
+        Y2 = fq.moe_grouped_linear(Xq_g, s_g, torch.from_numpy(offsets).cuda(), Wq, s_w)
+        torch.cuda.synchronize()
+    finally:
+        fq.set_gemm_tuning(0, 0, 0)
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_dispatch_moe_tokens(fq):
+    m = wl.moe()
+    row_token = np.asarray(m.token_of_row, dtype=np.int32)
+    T = m.X.shape[0]
+    got_q, got_s = run_dispatch(fq, m.X, wl.token_rows(row_token, T), len(row_token))
+    rows = sample_rows(len(row_token), 512, seed=14)
+    ref_q, ref_s = quant_rows(m.X.numpy()[row_token[rows]])
+    assert np.array_equal(got_q[rows], ref_q)
+    assert np.array_equal(got_s[rows].view(np.uint32), ref_s.view(np.uint32))
+    assert_no_device_error()

@@ -1,5 +1,6 @@
 """Checks of the seeded synthetic inputs and the FP16 top-2 router (harness only)."""
 import numpy as np
+import pytest
 import torch
 
 from fp8_quantized_generative_b200 import workloads as wl
@@ -67,3 +68,23 @@ def test_sweep_lognormal_signs():
     assert 0.45 < (x > 0).float().mean().item() < 0.55
     lm = x.abs().log()
     assert abs(lm.mean().item()) < 0.05 and 0.95 < lm.std().item() < 1.05
+
+
+def test_token_rows_inverts_the_grouping():
+    rng = np.random.default_rng(5)
+    T, E = 37, 6
+    logits = rng.standard_normal((T, E)).astype(np.float16)
+    row_token, _ = wl.group_by_expert(wl.route_top2(logits), E)
+    tr = wl.token_rows(row_token, T)
+    assert tr.shape == (T, 2) and tr.dtype == np.int32
+    # every grouped row appears exactly once, under its own token
+    flat = tr.reshape(-1)
+    assert np.array_equal(np.sort(flat[flat >= 0]), np.arange(len(row_token)))
+    for t in range(T):
+        for r in tr[t]:
+            assert r == -1 or row_token[r] == t
+    # a token with fewer rows than topk is padded with -1
+    tr1 = wl.token_rows(np.array([2, 0, 2]), 4)
+    assert tr1.tolist() == [[1, -1], [-1, -1], [0, 2], [-1, -1]]
+    with pytest.raises(ValueError):
+        wl.token_rows(np.array([1, 1, 1]), 2)

@@ -149,7 +149,7 @@ class Plan:
     """Device buffers (rotated sets) and the raw C-ABI launch sequence of one step."""
 
     def __init__(self, kind, tensors, device, min_rotation_bytes, fused=True, x_fmt="e4m3", weights="channel",
-                 dispatch="quant"):
+                 dispatch="quant", overlap=False):
         import fp8_quantized_generative_b200 as fq
         from fp8_quantized_generative_b200 import _lib
         self.fq, self.L = fq, _lib
@@ -167,6 +167,8 @@ class Plan:
         self.fmt = _lib.FORMATS[x_fmt]
         # Up to 16 token rows the library quantizes inside the GEMM (one launch; E4M3 only).
         self.fused = fused and kind == "dense" and x_fmt == "e4m3" and tensors[0].shape[0] <= fq.FUSED_MAX_ROWS
+        # More than 128 rows: one launch that quantizes inside the CTA-pair GEMM (E4M3 only).
+        self.overlap = overlap and kind == "dense" and x_fmt == "e4m3" and tensors[0].shape[0] > 128
         if kind == "dense":
             X, W = tensors
             self.M, self.K = X.shape
@@ -200,6 +202,9 @@ class Plan:
                 b["Xq"] = torch.empty((self.M, self.K), dtype=torch.uint8, device=device)
                 b["sx"] = torch.empty((self.M,), dtype=torch.float32, device=device)
                 b["Y"] = torch.empty((self.M, self.N), dtype=torch.float16, device=device)
+                if self.overlap:
+                    b["sync"] = torch.zeros((int(_lib.fp8q_overlap_sync_words(self.M)),), dtype=torch.int32,
+                                            device=device)
             else:
                 b["X"] = Xp.to(device)
                 b["off"] = torch.from_numpy(offsets).to(device)
@@ -230,6 +235,8 @@ class Plan:
     def _kernel_names(self):
         if self.fused:
             return ["fp8_quantized_linear_fused"]
+        if self.overlap:
+            return ["fp8_quantized_linear_overlapped"]
         if self.kind == "dense":
             return ["quant_rows", "fp8_gemm"]
         up = "fp8_grouped_gemm_up_gather" if self.gather else "fp8_grouped_gemm_up"
@@ -239,7 +246,7 @@ class Plan:
 
     def kernel_bytes_flops(self):
         """Algorithmic bytes and FLOPs of each launch of one step."""
-        if self.fused:
+        if self.fused or self.overlap:
             M, N, K = self.M, self.N, self.K
             return [(2 * M * K + N * K + 4 * N + 2 * M * N, 2.0 * M * N * K)]
         if self.kind == "dense":
@@ -267,6 +274,9 @@ class Plan:
         st = torch.cuda.current_stream(self.device).cuda_stream   # the capture stream inside a graph
         if self.fused:
             s = L.fp8q_quantized_linear(p["X"], p["Wq"], p["sw"], self.M, self.N, self.K, p["Y"], 0, 0, st)
+        elif self.overlap:
+            s = L.fp8q_quantized_linear_overlapped(p["X"], p["Wq"], p["sw"], self.M, self.N, self.K, p["Y"], p["Xq"],
+                                                   p["sx"], p["sync"], st)
         elif self.kind == "dense":
             if k == 0:
                 s = L.fp8q_quantize_rows_dynamic_fmt(p["X"], self.M, self.K, self.fmt, p["Xq"], p["sx"], st)
@@ -584,7 +594,7 @@ def run_ours(args, world, rank, local):
     import fp8_quantized_generative_b200 as fq
     fq.set_gemm_tuning({"auto": 0, "single": 1, "pair": 2, "splitk": 3}[args.gemm], args.bn, args.ksplit)
     plan = Plan(kind, tensors, device, min_rotation_bytes=3 * L2_BYTES, fused=args.fused, x_fmt=args.x_fmt,
-                dispatch=args.dispatch,
+                dispatch=args.dispatch, overlap=args.overlap,
                 weights=args.weight_scales)
     peaks, peak_src = load_peaks()
 
@@ -654,7 +664,7 @@ def run_ours(args, world, rank, local):
                        "l2": f"rotating {plan.sets} buffer sets of {plan.bytes_per_set / 1e6:.0f} MB "
                              f"(> 3x 126 MB L2), no flush",
                        "step": " -> ".join(plan.kernels),
-                       "fused": plan.fused,
+                       "fused": plan.fused, "overlap": plan.overlap,
                        "launch": "per-call from the host" if args.no_graph else
                                  "CUDA graph of the K timed steps (replayed once untimed to upload)",
                        "kernel_timing": "per-kernel: CUDA events around a graph of that kernel's K launches"
@@ -717,6 +727,8 @@ def main(argv=None):
     ap.add_argument("--fused", action="store_true",
                     help="one fused quantize+linear launch per step where it applies (<= 16 rows); "
                          "default: the two launches, measured faster on B200")
+    ap.add_argument("--overlap", action="store_true",
+                    help="M > 128: one launch per step that quantizes inside the CTA-pair GEMM")
     ap.add_argument("--gemm", default="auto", choices=["auto", "single", "pair", "splitk"],
                     help="dense GEMM kernel family (tuning sweeps; default: chosen per shape)")
     ap.add_argument("--bn", type=int, default=0, help="pair-kernel tile width (0 = automatic)")

@@ -27,7 +27,7 @@ from ._lib import Fp8qError, check, lib
 __all__ = [
     "Fp8qError", "lib", "quantize_rows_dynamic", "quantize_weight_per_channel", "quantize_weight_per_tensor",
     "quantize_weight_blockwise", "linear", "moe_grouped_linear", "moe_grouped_linear_gather",
-    "moe_grouped_linear_combine", "quantize_rows_dispatch",
+    "moe_grouped_linear_combine", "quantize_rows_dispatch", "quantized_linear_overlapped", "overlap_workspace",
     "moe_grouped_linear_blockscaled",
     "quantized_linear", "e4m3_encode_f32", "device_error", "set_gemm_tuning",
 ]
@@ -166,6 +166,38 @@ def quantized_linear(X: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
     s_x = torch.empty((M,), dtype=torch.float32, device=X.device)
     check(_lib.fp8q_quantized_linear(X.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K, Y.data_ptr(),
                                      Xq.data_ptr(), s_x.data_ptr(), _stream(X)), "fp8q_quantized_linear")
+    return Y
+
+
+def overlap_workspace(M: int, K: int, device) -> tuple:
+    """Workspace of quantized_linear_overlapped for M rows of K: (codes uint8
+    [M,K], scales fp32 [M], sync words int32, zero-filled).  Reusable across
+    calls that do not overlap on the GPU."""
+    words = int(_lib.fp8q_overlap_sync_words(M))
+    return (torch.empty((M, K), dtype=torch.uint8, device=device),
+            torch.empty((M,), dtype=torch.float32, device=device),
+            torch.zeros((words,), dtype=torch.int32, device=device))
+
+
+def quantized_linear_overlapped(X: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
+                                workspace: tuple | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """quantized_linear as one kernel for M > 128: the GEMM's own warps
+    quantize the rows while its tensor cores start on the rows already done.
+    The workspace (see overlap_workspace) then holds the codes and scales."""
+    _need(X, torch.float16, "X", 2)
+    _need(Wq, torch.uint8, "Wq", 2)
+    _need(s_w, torch.float32, "s_w", 1)
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or s_w.shape[0] != N:
+        raise ValueError("shape mismatch")
+    Xq, s_x, sync = workspace if workspace is not None else overlap_workspace(M, K, X.device)
+    if tuple(Xq.shape) != (M, K) or s_x.shape[0] != M or sync.numel() < _lib.fp8q_overlap_sync_words(M):
+        raise ValueError("workspace does not fit this X")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X.device)
+    check(_lib.fp8q_quantized_linear_overlapped(X.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K, Y.data_ptr(),
+                                                Xq.data_ptr(), s_x.data_ptr(), sync.data_ptr(), _stream(X)),
+          "fp8q_quantized_linear_overlapped")
     return Y
 
 

@@ -58,6 +58,8 @@ SIGNATURES = {
     "fp8q_linear_fmt": (_INT, [_P, _INT, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "fp8q_moe_grouped_linear_fmt": (_INT, [_P, _INT, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
     "fp8q_quantize_weight_blockwise": (_INT, [_P, _I32, _I64, _I64, _P, _P, _P]),
+    "fp8q_quantized_linear_overlapped": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
+    "fp8q_overlap_sync_words": (_I64, [_I64]),
     "fp8q_quantize_rows_dispatch": (_INT, [_P, _I64, _I64, _I32, _P, _I32, _I64, _P, _P, _P]),
     "fp8q_moe_grouped_linear_combine": (_INT, [_P, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P, _I64, _P, _P]),
     "fp8q_moe_grouped_linear_gather": (_INT, [_P, _P, _I64, _P, _P, _I32, _I64, _P, _P, _I64, _I64, _P, _P]),
@@ -148,6 +150,14 @@ def fp8q_moe_grouped_linear_fmt(Xq, x_fmt, s_x, offsets, E, rows, Wq, s_w, N, K,
 def fp8q_moe_grouped_linear_gather(Xq_tok, s_x_tok, tokens, row_token, offsets, E, rows, Wq, s_w, N, K, Y, stream):
     return lib().fp8q_moe_grouped_linear_gather(Xq_tok, s_x_tok, tokens, row_token, offsets, E, rows, Wq, s_w, N, K,
                                                 Y, stream)
+
+
+def fp8q_quantized_linear_overlapped(X, Wq, s_w, M, N, K, Y, Xq_ws, s_x_ws, sync_ws, stream):
+    return lib().fp8q_quantized_linear_overlapped(X, Wq, s_w, M, N, K, Y, Xq_ws, s_x_ws, sync_ws, stream)
+
+
+def fp8q_overlap_sync_words(M):
+    return lib().fp8q_overlap_sync_words(M)
 
 
 def fp8q_quantize_rows_dispatch(X, T, K, fmt, token_rows, topk, rows, Xq, s_x, stream):

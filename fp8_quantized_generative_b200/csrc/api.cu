@@ -328,7 +328,7 @@ TailSplit tail_split(int64_t full_tiles, int clusters, int bn) {
 // Launch a pair kernel.  Dense: A = Xq [rows, K], B = Wq [N, K].  Grouped:
 // B = Wq [E*N, K] and the schedule comes from the device offsets;
 // `tiles_upper_bound` caps the grid when the tile count is unknown on the host.
-template <int BN, int STAGES, bool kGrouped>
+template <int BN, int STAGES, bool kGrouped, bool kQuantA = false>
 fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, int64_t b_rows, const GemmParams& p0, int dev,
                         cudaStream_t st, int64_t tiles_upper_bound = 0) {
   using L = PairLayout<BN, STAGES>;
@@ -367,8 +367,8 @@ fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, int64_t b_rows, cons
   if (s != FP8Q_OK) return s;
   s = make_output_map(&ty, p.Y, p.rows, p.N);
   if (s != FP8Q_OK) return s;
-  auto kernel = fp8_gemm_pair_kernel<BN, STAGES, kGrouped>;
-  cudaError_t e = ensure_smem<fp8_gemm_pair_kernel<BN, STAGES, kGrouped>>(
+  auto kernel = fp8_gemm_pair_kernel<BN, STAGES, kGrouped, kQuantA>;
+  cudaError_t e = ensure_smem<fp8_gemm_pair_kernel<BN, STAGES, kGrouped, kQuantA>>(
       L::smem_bytes(kGrouped ? kMaxExperts : 0), dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair)");
   const int pairs = static_cast<int>(tiles < clusters ? (tiles < 1 ? 1 : tiles) : clusters);
@@ -755,6 +755,56 @@ fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const fl
   if (s != FP8Q_OK) return s;
   return fp8q_linear(Xq_ws, s_x_ws, Wq, s_w, M, N, K, Y_f16, stream);
 }
+
+fp8q_status fp8q_quantized_linear_overlapped(const void* X_f16, const uint8_t* Wq, const float* s_w, int64_t M,
+                                             int64_t N, int64_t K, void* Y_f16, uint8_t* Xq_ws, float* s_x_ws,
+                                             uint32_t* sync_ws, void* stream) {
+  if (M < 0 || M > kMaxDim) return invalid("M out of range");
+  if (N <= 0 || N > kMaxDim || N % 8 != 0) return invalid("N must be positive and a multiple of 8");
+  if (K <= 0 || K > kMaxDim || K % 16 != 0) return invalid("K must be positive and a multiple of 16");
+  if (M == 0) return FP8Q_OK;
+  if (!aligned16(X_f16) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y_f16) || !aligned16(Xq_ws) ||
+      !aligned16(s_x_ws) || !aligned16(sync_ws))
+    return invalid("null or non-16-byte-aligned pointer");
+  const Knobs kn = knobs();
+  // Up to 128 rows (split-K kernels) or with another kernel family forced:
+  // the two launches (the sync words are not touched).
+  if (M <= kBM || kn.force == 1 || kn.force == 3)
+    return fp8q_quantized_linear(X_f16, Wq, s_w, M, N, K, Y_f16, Xq_ws, s_x_ws, stream);
+  int dev = 0, sms = 0;
+  const cudaError_t e = current_device_info(&dev, &sms);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  GemmParams p = {};
+  p.s_x = s_x_ws;
+  p.s_w = s_w;
+  p.Y = static_cast<__half*>(Y_f16);
+  p.x_f16 = static_cast<const __half*>(X_f16);
+  p.q_out = Xq_ws;
+  p.s_out = s_x_ws;
+  p.sync = sync_ws;
+  p.rows = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.E = 1;
+  p.tail_q = 1;
+  p.x_fmt = FP8Q_FMT_E4M3;
+  // n-blocks first: the first round of tiles needs only the first row blocks,
+  // which the quantizing warps finish first.  FP8Q_RASTER = 1 overrides.
+  static const int raster = [] {
+    const char* v = std::getenv("FP8Q_RASTER");
+    return v ? std::atoi(v) : 0;
+  }();
+  p.n_fastest = raster == 1 ? 0 : 1;
+  const int clusters = max_pair_clusters<256, 6, false>(dev);
+  const int bn = kn.bn ? kn.bn : choose_pair_bn(M, N, clusters > 0 ? clusters : sms / 2);
+  switch (bn) {
+    case 128: return launch_pair<128, 8, false, true>(Xq_ws, Wq, N, p, dev, static_cast<cudaStream_t>(stream));
+    case 192: return launch_pair<192, 6, false, true>(Xq_ws, Wq, N, p, dev, static_cast<cudaStream_t>(stream));
+    default: return launch_pair<256, 6, false, true>(Xq_ws, Wq, N, p, dev, static_cast<cudaStream_t>(stream));
+  }
+}
+
+int64_t fp8q_overlap_sync_words(int64_t M) { return M < 0 ? 0 : qa_sync_words(M); }
 
 fp8q_status fp8q_quantized_linear_noalloc(const void* X_f16, const uint8_t* Wq, const float* s_w, int64_t M,
                                           int64_t N, int64_t K, void* Y_f16, void* stream) {

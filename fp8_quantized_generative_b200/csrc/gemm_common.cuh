@@ -50,6 +50,12 @@ struct GemmParams {
   int tokens;               // grouped gather / combine: rows of the token matrix
   const int32_t* comb_token; // combine: grouped row r adds into output row comb_token[r] (nullptr: plain store)
   const float* comb_weight;  // combine: the weight of grouped row r
+  // CTA-pair dense kernel with the activation quantization inside it: the
+  // codes and scales of x_f16 are written to q_out / s_out (= the A operand
+  // and s_x); sync holds the per-128-row-block ready flags.
+  uint8_t* q_out;
+  float* s_out;
+  uint32_t* sync;
 };
 
 // Row of the activation codes / scales that product row r reads (the row

@@ -20,9 +20,13 @@
 // second B descriptor with a narrower box), so the last round is short
 // instead of mostly idle.
 // No TMA multicast: every CTA loads only the tiles it stores.
+// kQuantA (dense): the kernel also quantizes the fp16 activations
+// (quant_in_gemm.cuh): the epilogue warps write the codes and scales, the
+// producer waits per 128-row block before loading them.
 #pragma once
 
 #include "gemm_fp8.cuh"
+#include "quant_in_gemm.cuh"
 
 namespace fp8q {
 
@@ -111,7 +115,7 @@ __device__ __forceinline__ PairTile pair_tile(int t, const GemmParams& p, int nu
   return r;
 }
 
-template <int BN, int STAGES, bool kGrouped>
+template <int BN, int STAGES, bool kGrouped, bool kQuantA = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAh,
                          const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBt,
@@ -119,6 +123,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   using L = PairLayout<BN, STAGES>;
   static_assert(BN % 64 == 0 && BN >= 64 && (BN <= 256 || BN == 512) && (BN / 2) % 8 == 0, "BN");
   static_assert(L::kNAcc * BN <= L::kTmemCols, "accumulators must fit in TMEM");
+  static_assert(!(kQuantA && kGrouped), "in-kernel quantization is the dense form");
   constexpr bool kWide = L::kWide;
   // A = activations: E4M3, or E5M2 for the activation-format variant
   const uint32_t kAFmt = idesc_a_fmt(p.x_fmt);
@@ -211,6 +216,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // The next kernel on the stream may begin launching (it waits for this
   // grid before touching anything this grid reads or writes).
   pdl_launch_dependents();
+  // In-kernel quantization, first pass: every warp of the grid one row.
+  const int qa_first = kQuantA ? qa_first_pass_rows(p, static_cast<int>(gridDim.x), kGemmThreads / 32) : 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -225,26 +232,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tma_load_2d_pair(dst, pt.tail ? &tmBt : &tmB, bar, kx, pt.b_row0 + static_cast<int>(rank) * (pt.bn / 2));
       }
     };
+    // The weights do not depend on the kernel launched before this one
+    // (programmatic dependent launch): request the first ring pass of the
+    // first tile's weight tiles before waiting for it; only the activation
+    // tiles wait.
+    int pre = 0;
+    if (lane == 0 && !kGrouped && pair < total) {
+      const PairTile pt = pair_tile<BN, kGrouped>(pair, p, num_m, num_n, tile_prefix, offs);
+      const uint32_t bytes = 2u * static_cast<uint32_t>(L::kABytes + (pt.bn / 2) * kBK);
+      pre = num_kb < STAGES ? num_kb : STAGES;
+      for (int i = 0; i < pre; ++i) {
+        const uint32_t full_leader = mapa_shared(smem_u32(&full[i]), 0);
+        if (leader) mbar_arrive_expect_tx(&full[i], bytes);
+        load_b(pt, sB + i * L::kBBytes, full_leader, i * kBK);
+      }
+    }
+    __syncwarp();
+    pdl_wait_prior_grid();
+    if (kQuantA)   // while those loads are in flight: this warp's row of the first pass
+      quantize_rows_strided(p, static_cast<int>(blockIdx.x) * (kGemmThreads / 32) + warp, 1 << 30, qa_first, lane);
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      // The weights do not depend on the kernel launched before this one
-      // (programmatic dependent launch): request the first ring pass of the
-      // first tile's weight tiles before waiting for it; only the activation
-      // tiles wait.
-      int pre = 0;
-      if (!kGrouped && pair < total) {
-        const PairTile pt = pair_tile<BN, kGrouped>(pair, p, num_m, num_n, tile_prefix, offs);
-        const uint32_t bytes = 2u * static_cast<uint32_t>(L::kABytes + (pt.bn / 2) * kBK);
-        pre = num_kb < STAGES ? num_kb : STAGES;
-        for (int i = 0; i < pre; ++i) {
-          const uint32_t full_leader = mapa_shared(smem_u32(&full[i]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[i], bytes);
-          load_b(pt, sB + i * L::kBBytes, full_leader, i * kBK);
-        }
-      }
-      pdl_wait_prior_grid();
+      RowsReady ready;
       for (int t = pair; t < total && ok; t += npairs) {
         const PairTile pt = pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs);
         // half tile: 64 rows of A per CTA (box of tmAh) at the start of the stage slot
@@ -252,6 +263,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int a_row = pt.a_row0 + static_cast<int>(rank) * a_rows;
         const CUtensorMap* tma_a = pt.half ? &tmAh : &tmA;
         const uint32_t bytes = 2u * static_cast<uint32_t>(a_rows * kBK + (pt.bn / 2) * kBK);
+        if (kQuantA && !ready.wait(p, a_row, true)) {   // this CTA's 128 rows quantized
+          ok = false;
+          break;
+        }
         for (int kb = 0; kb < num_kb; ++kb) {
           if (pre > 0) {
             // stage kb of the first pass: weights already requested
@@ -292,6 +307,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader CTA)
     pdl_wait_prior_grid();
+    if (kQuantA)
+      quantize_rows_strided(p, static_cast<int>(blockIdx.x) * (kGemmThreads / 32) + warp, 1 << 30, qa_first, lane);
     if (lane == 0 && leader) {
       int s = 0, acc = 0;
       uint32_t ph = 0, acc_ph = 0;
@@ -349,11 +366,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     pdl_wait_prior_grid();   // s_x comes from, and Y may be read by, the neighbouring kernels
+    if (kQuantA) {
+      // the first pass (one row per warp of the grid), then the rest over the epilogue warps
+      quantize_rows_strided(p, static_cast<int>(blockIdx.x) * (kGemmThreads / 32) + warp, 1 << 30, qa_first, lane);
+      quantize_rows_strided(p, qa_first + static_cast<int>(blockIdx.x) * kEpiWarps + (warp - kEpiWarp0),
+                            static_cast<int>(gridDim.x) * kEpiWarps, p.rows, lane);
+    }
     uint8_t* stage = sEpi + (warp - kEpiWarp0) * kStageTileBytes;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     int acc = 0;
     uint32_t acc_ph = 0;
+    RowsReady ready;
     for (int t = pair; t < total; t += npairs) {
       const PairTile pt = pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs);
       EpiTile et;
@@ -363,7 +387,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       et.sw0 = pt.sw0;
       et.clip = !kGrouped;   // dense: rows past the end are past the tensor
       const EpiWarpView wv = epi_view(et, warp, pt.bn, pt.half);
-      const EpiScales<BN / 64> sc = epilogue_scales<BN / 64>(et, p, wv, lane);
+      EpiScales<BN / 64> sc = epilogue_scales<BN / 64>(et, p, wv, lane);
+      if (kQuantA) {
+        // the row scales were written in this kernel: read them once the
+        // block is complete (it is before its first MMA, so this wait ends)
+        if (!ready.wait(p, et.row0, false)) {
+          raise_error(0x4u);
+          *abort_flag = 1;
+          break;
+        }
+        const int r = wv.qrow0 + lane;
+        sc.sx = r < et.row_end ? ld_relaxed_gpu_f32(p.s_x + r) : 0.0f;
+      }
       if (!mbar_wait(&tfull[acc], acc_ph, abort_flag)) {
         raise_error(0x4u);
         *abort_flag = 1;
@@ -385,6 +420,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 
   __syncthreads();
+  if (kQuantA && threadIdx.x == 0) release_sync(p);   // after every read of the flags in this CTA
   // The leader has drained its MMAs (which read both CTAs' shared memory) and
   // all cross-CTA arrivals were issued before this point.
   tc_fence_before();

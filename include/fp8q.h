@@ -130,6 +130,28 @@ fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const fl
                                   uint8_t* Xq_ws, float* s_x_ws, void* stream);
 
 /*
+ * fp8q_quantized_linear as ONE kernel for M > 128 rows  [P2 §2.3: the
+ * QuantizeLinear + GEMM + Dequantize fusion]: the CTA-pair GEMM's epilogue
+ * warps quantize the fp16 rows (same steps, codes and scales as
+ * fp8q_quantize_rows_dynamic) into Xq_ws [M,K] uint8 / s_x_ws [M] fp32 while
+ * its tensor cores start on the 128-row blocks already published; Y as
+ * fp8q_quantized_linear.  sync_ws: uint32 [fp8q_overlap_sync_words(M)],
+ * device, ZERO-FILLED before the first call; every call that completes
+ * leaves it zero again.  Calls sharing one sync_ws must not overlap on the
+ * GPU; after a device error (fp8q_device_error() != 0) zero it again.  With
+ * M <= 128 the call runs the two-step path of fp8q_quantized_linear
+ * (sync_ws untouched).  All pointers 16-byte aligned.
+ */
+fp8q_status fp8q_quantized_linear_overlapped(const void* X_f16, const uint8_t* Wq, const float* s_w,
+                                             int64_t M, int64_t N, int64_t K, void* Y_f16,
+                                             uint8_t* Xq_ws, float* s_x_ws, uint32_t* sync_ws,
+                                             void* stream);
+
+/* Number of uint32 words fp8q_quantized_linear_overlapped needs in sync_ws
+ * for M rows: 2 + 2 * ceil(M / 128). */
+int64_t fp8q_overlap_sync_words(int64_t M);
+
+/*
  * Allocation-free form of fp8q_quantized_linear (the pages have no
  * counterpart; this is a deployment convenience).  Same inputs, output and
  * numerics as fp8q_quantized_linear with a workspace, but the codes and

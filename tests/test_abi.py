@@ -199,3 +199,18 @@ def test_dispatch_rejects(L):
     assert d(a, 4, 32, 0, a, 2, 8, BAD, a, 0) == _lib.FP8Q_ERR_INVALID_ARG    # Xq alignment
     assert d(a, 4, 32, 0, a, 2, 0, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG      # tokens, no rows
     assert d(0, 0, 32, 0, 0, 2, 0, 0, 0, 0) == _lib.FP8Q_OK                   # nothing to do
+
+
+def test_overlapped_rejects_and_sync_words(L):
+    a = 0x1000
+    o = _lib.fp8q_quantized_linear_overlapped
+    #      X  Wq sw M    N   K   Y  Xq sx sync st
+    assert o(a, a, a, 300, 12, 32, a, a, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG     # N % 8
+    assert o(a, a, a, 300, 16, 24, a, a, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG     # K % 16
+    assert o(a, a, a, 300, 16, 32, a, a, a, 0, 0) == _lib.FP8Q_ERR_INVALID_ARG     # null sync
+    assert o(a, a, a, 300, 16, 32, a, a, a, BAD, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert o(a, a, a, 300, 16, 32, a, BAD, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert o(a, a, a, -1, 16, 32, a, a, a, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert o(0, 0, 0, 0, 16, 32, 0, 0, 0, 0, 0) == _lib.FP8Q_OK                     # M = 0
+    w = _lib.fp8q_overlap_sync_words
+    assert [w(0), w(1), w(128), w(129), w(4096)] == [2, 4, 4, 6, 66]

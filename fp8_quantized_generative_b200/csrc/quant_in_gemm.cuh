@@ -91,8 +91,6 @@ __device__ __forceinline__ void quantize_rows_strided(const GemmParams& p, int r
   if (done > 0 && lane == 0) red_release_gpu_add(p.sync + 1, done);
 }
 
-
-
 // Rows of the first pass: one per warp of the grid (all warps of every CTA).
 __device__ __forceinline__ int qa_first_pass_rows(const GemmParams& p, int ncta, int warps_per_cta) {
   const int n = ncta * warps_per_cta;

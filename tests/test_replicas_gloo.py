@@ -51,3 +51,23 @@ def test_reference_arm_runs_only_on_rank_zero(monkeypatch):
     class A:
         workload, steps, warmup, gpus = "tiny", 1, 0, 2
     assert bench.run_reference(A, world=2, rank=1) is None
+
+
+@pytest.mark.parametrize("workload", ["tiny", "moe_tokens"])
+def test_reference_arm_line_on_rank_zero(workload):
+    # the reference arm is the CPU oracle on a bounded sample of the workload;
+    # its line carries the contract's keys and a cpu_baseline describing itself
+    class A:
+        steps, warmup, gpus = 2, 1, 1
+        x_fmt, weight_scales = "e4m3", "channel"
+    A.workload = workload
+    line = bench.run_reference(A, world=1, rank=0)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["config"]["workload"].startswith(bench.workload_spec(workload)[0][:10])

@@ -921,12 +921,13 @@ fp8q_status fp8q_moe_grouped_linear_combine(const uint8_t* Xq, const float* s_x,
   if (rows > 0 && (row_weight == nullptr || (reinterpret_cast<uintptr_t>(row_weight) & 3u) != 0))
     return invalid("row_weight pointer");
   if (!aligned16(out_f16)) return invalid("null or non-16-byte-aligned output");
+  // every check before the output is touched (with no rows, the row-side pointers may be null)
+  if (rows > 0 && (!aligned16(Xq) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_w)))
+    return invalid("null or non-16-byte-aligned pointer");
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(out_f16, 0, static_cast<size_t>(tokens * N) * sizeof(__half), st);
   if (e != cudaSuccess) return cuda_fail(e, "combine output clear");
-  if (rows == 0) return FP8Q_OK;   // every row-side pointer may be null
-  if (!aligned16(Xq) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_w))
-    return invalid("null or non-16-byte-aligned pointer");
+  if (rows == 0) return FP8Q_OK;
   GemmParams p = {};   // every field set below; zero for the rest
   p.s_x = s_x;
   p.s_w = s_w;

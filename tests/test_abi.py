@@ -214,3 +214,11 @@ def test_overlapped_rejects_and_sync_words(L):
     assert o(0, 0, 0, 0, 16, 32, 0, 0, 0, 0, 0) == _lib.FP8Q_OK                     # M = 0
     w = _lib.fp8q_overlap_sync_words
     assert [w(0), w(1), w(128), w(129), w(4096)] == [2, 4, 4, 6, 66]
+
+
+def test_combine_rejects_misaligned_operands_before_touching_the_output(L):
+    # with rows > 0, a misaligned operand is rejected on the host (no memset is queued)
+    a = 0x1000
+    c = _lib.fp8q_moe_grouped_linear_combine
+    assert c(BAD, a, a, 4, 8, a, a, 16, 32, a, a, 4, a, 0) == _lib.FP8Q_ERR_INVALID_ARG
+    assert c(a, a, a, 4, 8, BAD, a, 16, 32, a, a, 4, a, 0) == _lib.FP8Q_ERR_INVALID_ARG

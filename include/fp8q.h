@@ -57,7 +57,7 @@ extern "C" {
 typedef enum {
   FP8Q_OK = 0,
   FP8Q_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment       */
-  FP8Q_ERR_UNSUPPORTED = 2,   /* valid request this build cannot serve      */
+  FP8Q_ERR_UNSUPPORTED = 2,   /* valid request this library cannot serve    */
   FP8Q_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed          */
   FP8Q_ERR_TIMEOUT = 4,       /* a device wait ran out (fp8q_device_error)  */
   FP8Q_ERR_DEVICE_CHECK = 5   /* a device-side input check failed           */

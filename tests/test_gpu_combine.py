@@ -193,3 +193,29 @@ def test_moe_down_combine(fq):
     S = magnitude_sum(xq, sx, sub_off, wq, sw, tok_local, m.row_weight[pick], len(toks))
     assert_close_combine(to_np(out)[toks], ref, S, "moe down combine")
     assert_no_device_error()
+
+
+def test_hand_worked_fixture_bit_exact(fq):
+    # tests/golden/moe_combine_hand.json: every intermediate is exact, so the
+    # GPU result must equal the hand-derived values bit for bit (channels 2..7
+    # have zero weights and stay zero: the API wants N % 8 == 0)
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "moe_combine_hand.json")))
+    R, K, E, N = len(g["row_token"]), g["K"], g["E"], 8
+    Xq = torch.zeros((R, K), dtype=torch.uint8)
+    Xq[:, 0] = torch.tensor(g["x_code_k0"], dtype=torch.uint8)
+    Wq = torch.zeros((E, N, K), dtype=torch.uint8)
+    Wq[:, :2, 0] = torch.tensor(g["w_code_k0"], dtype=torch.uint8)
+    s_w = torch.ones((E, N), dtype=torch.float32)
+    s_w[:, :2] = torch.tensor(g["s_w"], dtype=torch.float32)
+    out = fq.moe_grouped_linear_combine(
+        Xq.cuda(), torch.tensor(g["s_x"], dtype=torch.float32).cuda(),
+        torch.tensor(g["offsets"], dtype=torch.int32).cuda(), Wq.cuda(), s_w.cuda(),
+        torch.tensor(g["row_token"], dtype=torch.int32).cuda(), torch.tensor(g["row_weight"], dtype=torch.float32).cuda(),
+        g["tokens"])
+    torch.cuda.synchronize()
+    exp = np.zeros((g["tokens"], N), np.float16)
+    exp[:, :2] = np.array(g["expected"], np.float16)
+    assert np.array_equal(to_np(out).view(np.uint16), exp.view(np.uint16))
+    assert_no_device_error()

@@ -318,3 +318,21 @@ def test_combine_is_within_fp16_rounding_of_the_weighted_sum():
     np.add.at(mag, row_token, np.abs(row_w[:, None].astype(np.float64) * Y.astype(np.float64)))
     # three fp16 roundings (each row's y, each contribution, the sum): <= 2^-10 of the magnitudes
     assert np.all(np.abs(out - exact) <= 2.0 ** -10 * (mag + np.abs(exact)) + 2.0 ** -24)
+
+
+def test_combine_hand_worked_fixture():
+    """tests/golden/moe_combine_hand.json: values derived by hand (exact in fp16)."""
+    import json
+    import os
+    from oracle import moe_combine_ref
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "moe_combine_hand.json")))
+    R, K = len(g["row_token"]), g["K"]
+    Xq = np.zeros((R, K), np.uint8)
+    Xq[:, 0] = g["x_code_k0"]
+    Wq = np.zeros((g["E"], g["N"], K), np.uint8)
+    Wq[:, :, 0] = g["w_code_k0"]
+    out = moe_combine_ref(Xq, np.array(g["s_x"], np.float32), np.array(g["offsets"]), Wq,
+                          np.array(g["s_w"], np.float32), np.array(g["row_token"]),
+                          np.array(g["row_weight"], np.float32), g["tokens"])
+    assert out.dtype == np.float16
+    np.testing.assert_array_equal(out.astype(np.float64), np.array(g["expected"], np.float64))

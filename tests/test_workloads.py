@@ -88,3 +88,21 @@ def test_token_rows_inverts_the_grouping():
     assert tr1.tolist() == [[1, -1], [-1, -1], [0, 2], [-1, -1]]
     with pytest.raises(ValueError):
         wl.token_rows(np.array([1, 1, 1]), 2)
+
+
+def test_gate_weights_and_row_weights():
+    # softmax over each token's selected logits, highest logit first; the row
+    # weights follow the grouped-row order of group_by_expert
+    logits = np.array([[0.0, 1.0, -1.0, 2.0], [3.0, 3.0, 0.0, -2.0]], np.float16)
+    experts = wl.route_top2(logits)
+    assert experts.tolist() == [[3, 1], [0, 1]]
+    g = wl.gate_weights(logits, experts)
+    e = 1.0 / (1.0 + np.exp(-1.0))                 # softmax of (2, 1): e^2 / (e^2 + e^1)
+    np.testing.assert_allclose(g[0], [e, 1 - e], rtol=1e-6)
+    np.testing.assert_allclose(g[1], [0.5, 0.5], rtol=1e-6)     # equal logits
+    assert g.dtype == np.float32 and np.allclose(g.sum(axis=1), 1.0)
+    row_token, offsets = wl.group_by_expert(experts, 4)
+    rw = wl.row_weights(g, experts)
+    # grouped rows: expert 0: token 1; expert 1: tokens 0, 1; expert 3: token 0
+    assert row_token.tolist() == [1, 0, 1, 0] and list(offsets) == [0, 1, 3, 3, 4]
+    np.testing.assert_allclose(rw, [g[1, 0], g[0, 1], g[1, 1], g[0, 0]], rtol=0)

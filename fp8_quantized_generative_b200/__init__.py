@@ -93,15 +93,15 @@ def quantize_rows_dispatch(X: torch.Tensor, token_rows: torch.Tensor, rows: int,
     return Xq, s
 
 
-def quantize_weight_per_channel(W: torch.Tensor):
+def quantize_weight_per_channel(W: torch.Tensor, out: tuple | None = None):
     """Offline per-output-channel E4M3 quantization: fp16 [N,K] or [E,N,K]."""
     _need(W, torch.float16, "W")
     if W.dim() not in (2, 3):
         raise ValueError("W must be [N,K] or [E,N,K]")
     K = W.shape[-1]
     rows = W.numel() // K
-    Wq = torch.empty(W.shape, dtype=torch.uint8, device=W.device)
-    s = torch.empty(W.shape[:-1], dtype=torch.float32, device=W.device)
+    Wq, s = out if out is not None else (torch.empty(W.shape, dtype=torch.uint8, device=W.device),
+                                         torch.empty(W.shape[:-1], dtype=torch.float32, device=W.device))
     check(_lib.fp8q_quantize_weight_per_channel(W.data_ptr(), rows, K, Wq.data_ptr(), s.data_ptr(), _stream(W)),
           "fp8q_quantize_weight_per_channel")
     return Wq, s

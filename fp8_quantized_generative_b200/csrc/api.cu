@@ -545,15 +545,17 @@ fp8q_status check_quant_args(const void* X, int64_t M, int64_t K, const void* Q,
 
 bool valid_fmt(int fmt) { return fmt == FP8Q_FMT_E4M3 || fmt == FP8Q_FMT_E5M2; }
 
+// weights = true: the kernel lets the next one start only when it has
+// finished (the GEMMs read weight tiles before their dependency wait).
 fp8q_status quantize(const void* X, int64_t M, int64_t K, uint8_t* Q, float* S, void* stream,
-                     int fmt = FP8Q_FMT_E4M3) {
+                     int fmt = FP8Q_FMT_E4M3, bool weights = false) {
   fp8q_status s = check_quant_args(X, M, K, Q, S);
   if (s != FP8Q_OK || M == 0) return s;
   const __half* Xh = static_cast<const __half*>(X);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const cudaError_t e = fmt == FP8Q_FMT_E5M2
-                            ? launch_quant_rows<kFmtE5M2>(Xh, static_cast<int>(M), static_cast<int>(K), Q, S, st)
-                            : launch_quant_rows<kFmtE4M3>(Xh, static_cast<int>(M), static_cast<int>(K), Q, S, st);
+  const int m = static_cast<int>(M), k = static_cast<int>(K);
+  const cudaError_t e = fmt == FP8Q_FMT_E5M2 ? launch_quant_rows<kFmtE5M2>(Xh, m, k, Q, S, st, RowDispatch{}, !weights)
+                                             : launch_quant_rows<kFmtE4M3>(Xh, m, k, Q, S, st, RowDispatch{}, !weights);
   if (e != cudaSuccess) return cuda_fail(e, "quant_rows launch");
   return FP8Q_OK;
 }
@@ -650,7 +652,7 @@ fp8q_status fp8q_quantize_rows_dynamic(const void* X_f16, int64_t M, int64_t K, 
 fp8q_status fp8q_quantize_weight_per_channel(const void* W_f16, int64_t N, int64_t K, uint8_t* Wq, float* s_w,
                                              void* stream) {
   if (N == 0) return invalid("N must be positive");
-  return quantize(W_f16, N, K, Wq, s_w, stream);
+  return quantize(W_f16, N, K, Wq, s_w, stream, FP8Q_FMT_E4M3, true);
 }
 
 fp8q_status fp8q_quantize_rows_dynamic_fmt(const void* X_f16, int64_t M, int64_t K, fp8q_format fmt, uint8_t* Xq,

@@ -312,7 +312,8 @@ __global__ void __maxnreg__(96)
 __global__ void __launch_bounds__(256) quant_blocks_kernel(const __half* __restrict__ W, int N, int K, int NB,
                                                           int KB, uint8_t* __restrict__ Q, float* __restrict__ S) {
   __shared__ float red[8];
-  pdl_launch_dependents();
+  // Weights: the next kernel starts only once this one has finished (the
+  // GEMMs request weight tiles before their programmatic-dependent wait).
   pdl_wait_prior_grid();
   const int e = blockIdx.x / NB;
   const int bi = blockIdx.x - e * NB;

@@ -107,12 +107,14 @@ __device__ __forceinline__ void store_row_codes(const RowDispatch& d, int row, i
 template <int TPR, int VPT, int F, int CTA = 256>
 __global__ void __launch_bounds__(CTA) quant_rows_kernel(const __half* __restrict__ X, int M, int K,
                                                         uint8_t* __restrict__ Q, float* __restrict__ S,
-                                                        const RowDispatch d) {
+                                                        const RowDispatch d, const bool release_early) {
   static_assert(TPR >= 32 && TPR <= CTA && CTA <= 256 && (TPR & (TPR - 1)) == 0, "TPR");
   // Programmatic dependent launch: let the next kernel start its set-up now
   // (it waits for this grid before touching our outputs), and wait for the
-  // previous kernel before reading X or writing Q and S.
-  pdl_launch_dependents();
+  // previous kernel before reading X or writing Q and S.  Not for weights:
+  // the GEMMs request weight tiles before their own wait, so a weight
+  // quantization lets the next kernel start only once it has finished.
+  if (release_early) pdl_launch_dependents();
   pdl_wait_prior_grid();
   constexpr int kRowsPerCta = CTA / TPR;
   constexpr int kWarpsPerRow = TPR / 32;
@@ -160,9 +162,9 @@ __global__ void __launch_bounds__(CTA) quant_rows_kernel(const __half* __restric
 template <int F>
 __global__ void __launch_bounds__(256) quant_rows_long_kernel(const __half* __restrict__ X, int M, int K,
                                                              uint8_t* __restrict__ Q, float* __restrict__ S,
-                                                             const RowDispatch d) {
+                                                             const RowDispatch d, const bool release_early) {
   __shared__ float red[8];
-  pdl_launch_dependents();
+  if (release_early) pdl_launch_dependents();
   pdl_wait_prior_grid();
   const int row = blockIdx.x;
   const int nvec = K >> 3;
@@ -205,11 +207,13 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const __half* __re
 //                        into S[row] for rows >= 1 (S[0] is still being read);
 //   quant_tensor_finish  S[0] = s.
 // The scale is thus replicated once per row (output channel), the form the
-// per-channel GEMM epilogue consumes.
+// per-channel GEMM epilogue consumes.  These kernels quantize weights only, so
+// none lets the next kernel start early: the GEMMs request weight tiles before
+// their programmatic-dependent-launch wait, which is safe only because every
+// kernel writing weights has finished before the next kernel starts.
 __global__ void __launch_bounds__(256) tensor_amax_kernel(const __half* __restrict__ X, int64_t nvec,
                                                          unsigned int* __restrict__ amax_bits) {
   __shared__ float red[8];
-  pdl_launch_dependents();
   pdl_wait_prior_grid();
   const uint4* src = reinterpret_cast<const uint4*>(X);
   float m = 0.0f;
@@ -229,7 +233,6 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const __half* __restri
 
 __global__ void __launch_bounds__(256) quant_tensor_kernel(const __half* __restrict__ X, int M, int64_t nvec,
                                                           uint8_t* __restrict__ Q, float* __restrict__ S) {
-  pdl_launch_dependents();
   pdl_wait_prior_grid();
   const RowScale rs = row_scale_from_amax<kFmtE4M3>(S[0]);
   const uint4* src = reinterpret_cast<const uint4*>(X);
@@ -241,7 +244,6 @@ __global__ void __launch_bounds__(256) quant_tensor_kernel(const __half* __restr
 }
 
 __global__ void quant_tensor_finish_kernel(float* __restrict__ S) {
-  pdl_launch_dependents();
   pdl_wait_prior_grid();
   if (threadIdx.x == 0 && blockIdx.x == 0) S[0] = row_scale_from_amax<kFmtE4M3>(S[0]).s;
 }
@@ -279,14 +281,16 @@ inline cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cu
 }
 
 // Host-side launcher: picks (TPR, VPT) so one row fits in registers.
+// release_early = false for weights (see quant_rows_kernel).
 template <int F = kFmtE4M3>
 inline cudaError_t launch_quant_rows(const __half* X, int M, int K, uint8_t* Q, float* S, cudaStream_t st,
-                                     const RowDispatch d = RowDispatch{}) {
+                                     const RowDispatch d = RowDispatch{}, const bool release_early = true) {
   const int nvec = K / 8;
   int tpr = 32;
   while (tpr < 256 && tpr * 8 < nvec) tpr *= 2;
   const int vpt_needed = (nvec + tpr - 1) / tpr;
-  if (vpt_needed > 8) return launch_pdl(quant_rows_long_kernel<F>, dim3(M), dim3(256), st, X, M, K, Q, S, d);
+  if (vpt_needed > 8)
+    return launch_pdl(quant_rows_long_kernel<F>, dim3(M), dim3(256), st, X, M, K, Q, S, d, release_early);
   const int vpt = vpt_needed <= 1 ? 1 : vpt_needed <= 2 ? 2 : vpt_needed <= 4 ? 4 : 8;
   // Few rows (fewer than 256 CTAs of 256 threads, i.e. under ~2 per SM):
   // CTAs of 64 threads spread them over more SMs (measured 10% faster at
@@ -298,8 +302,9 @@ inline cudaError_t launch_quant_rows(const __half* X, int M, int K, uint8_t* Q, 
   const dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
 #define FP8Q_QR_CASE(T, V)                                                                                      \
   if (tpr == T && vpt == V)                                                                                   \
-    return small ? launch_pdl(quant_rows_kernel<T, V, F, (T < 64 ? 64 : T)>, grid, dim3(cta), st, X, M, K, Q, S, d) \
-                 : launch_pdl(quant_rows_kernel<T, V, F, 256>, grid, dim3(cta), st, X, M, K, Q, S, d);
+    return small ? launch_pdl(quant_rows_kernel<T, V, F, (T < 64 ? 64 : T)>, grid, dim3(cta), st, X, M, K, Q, S, d, \
+                              release_early)                                                                  \
+                 : launch_pdl(quant_rows_kernel<T, V, F, 256>, grid, dim3(cta), st, X, M, K, Q, S, d, release_early);
   FP8Q_QR_CASE(32, 1) FP8Q_QR_CASE(32, 2) FP8Q_QR_CASE(32, 4) FP8Q_QR_CASE(32, 8)
   FP8Q_QR_CASE(64, 8) FP8Q_QR_CASE(128, 8) FP8Q_QR_CASE(256, 8)
 #undef FP8Q_QR_CASE

@@ -34,13 +34,58 @@ def assert_close_f16(y_gpu, y_ref, what=""):
         assert rel <= REL_FRO, f"{what}: relative Frobenius error {rel:.3e} > {REL_FRO}"
 
 
-def sample_rows(M, n, seed=0):
-    """Up to n row indices spread over [0, M): always the first and last rows."""
-    if M <= n:
-        return np.arange(M)
-    rng = np.random.default_rng(seed)
-    mid = rng.choice(np.arange(1, M - 1), size=n - 2, replace=False)
-    return np.sort(np.concatenate([[0, M - 1], mid]))
+class Guarded:
+    """A device tensor placed in the middle of a larger byte buffer whose
+    `pad` bytes on either side hold a seeded byte pattern.
+
+    Stands in for a memory checker: a kernel that writes past either end of
+    the tensor changes the pattern, and check() reports it.  The interior
+    starts `pad` bytes (a multiple of 256) into the allocation, so it keeps
+    the 16-byte alignment the library requires.
+    """
+
+    def __init__(self, shape, dtype, fill=None, pad=4096, seed=0, device="cuda"):
+        assert pad % 256 == 0
+        self.pad = pad
+        esize = torch.empty((), dtype=dtype).element_size()
+        n = int(np.prod(shape)) if len(shape) else 1
+        self.nbytes = n * esize
+        g = torch.Generator().manual_seed(1000 + seed)
+        total = 2 * pad + self.nbytes
+        self.pattern = torch.randint(0, 256, (total,), generator=g, dtype=torch.uint8).to(device)
+        self.buf = self.pattern.clone()
+        inner = self.buf[pad:pad + self.nbytes]
+        self.t = inner.view(dtype).view(shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def check(self, what=""):
+        lo = self.buf[:self.pad]
+        hi = self.buf[self.pad + self.nbytes:]
+        for name, got, exp in (("before", lo, self.pattern[:self.pad]),
+                               ("after", hi, self.pattern[self.pad + self.nbytes:])):
+            bad = (got != exp).nonzero()
+            if bad.numel():
+                first = int(bad[0, 0]) if name == "after" else int(bad[-1, 0]) - self.pad
+                raise AssertionError(f"{what}: {bad.numel()} guard bytes {name} the tensor were overwritten "
+                                     f"(nearest at byte offset {first} from its {'end' if name == 'after' else 'start'})")
+
+
+class Guards:
+    """Factory of Guarded tensors that checks all of them at once."""
+
+    def __init__(self):
+        self.items = []
+
+    def __call__(self, shape, dtype, fill=None, name=""):
+        g = Guarded(tuple(shape), dtype, fill, seed=len(self.items))
+        self.items.append((name or f"tensor {len(self.items)}", g))
+        return g.t
+
+    def check(self, what=""):
+        torch.cuda.synchronize()
+        for name, g in self.items:
+            g.check(f"{what} {name}".strip())
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:

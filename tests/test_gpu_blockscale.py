@@ -6,7 +6,7 @@ block-aligned MoE quantization, activations per token).
   oracle.quant_blocks, per expert (blocks never span experts);
 * fp8q_moe_grouped_linear_blockscaled: FP16 outputs within the path's
   tolerance of oracle.moe_blockscaled_ref on ragged groups, adversarial
-  offsets and the MoE configuration (sampled rows).
+  offsets and the full MoE configuration (every row; guard-banded output).
 """
 import numpy as np
 import pytest
@@ -15,7 +15,7 @@ import torch
 from oracle import linear_blockscaled_ref, moe_blockscaled_ref, quant_blocks, quant_rows
 from fp8_quantized_generative_b200 import workloads as wl
 
-from parity import assert_close_f16, assert_no_device_error, sample_rows, to_np
+from parity import Guards, assert_close_f16, assert_no_device_error, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -53,9 +53,10 @@ def run_bs(fq, X, offsets, W):
     Wq, s_wb = fq.quantize_weight_blockwise(W.cuda())
     Xq, s_x = fq.quantize_rows_dynamic(X.cuda())
     off = torch.from_numpy(np.asarray(offsets, dtype=np.int32)).cuda()
-    Y = torch.full((X.shape[0], W.shape[1]), float("nan"), dtype=torch.float16, device="cuda")
+    g = Guards()
+    Y = g((X.shape[0], W.shape[1]), torch.float16, float("nan"), "Y")
     fq.moe_grouped_linear_blockscaled(Xq, s_x, off, Wq, s_wb, out=Y)
-    torch.cuda.synchronize()
+    g.check("block-scaled")
     return Y
 
 
@@ -125,8 +126,8 @@ def moe_case():
 def test_moe_up_blockscaled(fq, moe_case):
     m = moe_case
     Y = run_bs(fq, m.X_perm, m.offsets, m.W_up)
-    rows = sample_rows(m.X_perm.shape[0], 192, seed=6)
-    assert_close_f16(to_np(Y)[rows], oracle_rows_bs(m.X_perm, m.offsets, m.W_up, rows), "block-scaled moe up")
+    rows = np.arange(m.X_perm.shape[0])            # every grouped row
+    assert_close_f16(to_np(Y), oracle_rows_bs(m.X_perm, m.offsets, m.W_up, rows), "block-scaled moe up")
     assert_no_device_error()
 
 
@@ -134,6 +135,6 @@ def test_moe_down_blockscaled(fq, moe_case):
     m = moe_case
     Xd = wl.random_f16((m.X_perm.shape[0], wl.MOE_F), seed=304)
     Y = run_bs(fq, Xd, m.offsets, m.W_down)
-    rows = sample_rows(Xd.shape[0], 192, seed=7)
-    assert_close_f16(to_np(Y)[rows], oracle_rows_bs(Xd, m.offsets, m.W_down, rows), "block-scaled moe down")
+    rows = np.arange(Xd.shape[0])                  # every grouped row
+    assert_close_f16(to_np(Y), oracle_rows_bs(Xd, m.offsets, m.W_down, rows), "block-scaled moe down")
     assert_no_device_error()

@@ -11,7 +11,7 @@ import torch
 from oracle import moe_gather_ref, quant_rows
 from fp8_quantized_generative_b200 import workloads as wl
 
-from parity import assert_close_f16, assert_no_device_error, sample_rows, to_np
+from parity import Guards, assert_close_f16, assert_no_device_error, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -32,10 +32,11 @@ def routed(T, E, seed):
 def run_gather(fq, X, row_token, offsets, W):
     Xq, s_x = fq.quantize_rows_dynamic(X.cuda())
     Wq, s_w = fq.quantize_weight_per_channel(W.cuda())
-    Y = torch.full((len(row_token), W.shape[1]), float("nan"), dtype=torch.float16, device="cuda")
+    g = Guards()
+    Y = g((len(row_token), W.shape[1]), torch.float16, float("nan"), "Y")
     fq.moe_grouped_linear_gather(Xq, s_x, torch.from_numpy(row_token).cuda(), torch.from_numpy(offsets).cuda(),
                                  Wq, s_w, out=Y)
-    torch.cuda.synchronize()
+    g.check("gather")
     return Y, (Xq, s_x, Wq, s_w)
 
 
@@ -84,32 +85,25 @@ def test_bad_token_index_is_reported(fq):
 
 
 def test_moe_up_from_tokens(fq):
+    # every grouped row of the full-size up projection read from the token matrix
     m = wl.moe()
     row_token = np.asarray(m.token_of_row, dtype=np.int32)
     offsets = np.asarray(m.offsets, dtype=np.int32)
     Y, _ = run_gather(fq, m.X, row_token, offsets, m.W_up)
-    rows = sample_rows(len(row_token), 256, seed=12)
-    E, N, K = m.W_up.shape
-    # oracle on the sampled rows only (quantize the sampled tokens; each row with its expert)
-    expert_of = np.searchsorted(offsets.astype(np.int64), rows, side="right") - 1
-    xq, sx = quant_rows(m.X.numpy()[row_token[rows]])
-    ref = np.zeros((len(rows), N), np.float16)
-    from oracle import linear_ref
-    for e in np.unique(expert_of):
-        sel = expert_of == e
-        wq, sw = quant_rows(m.W_up[e].numpy())
-        ref[sel] = linear_ref(xq[sel], sx[sel], wq, sw)
-    assert_close_f16(to_np(Y)[rows], ref, "moe up from tokens")
+    assert_close_f16(to_np(Y), oracle_gather(m.X, row_token, offsets, m.W_up), "moe up from tokens")
     assert_no_device_error()
 
 
 # ------------------------------------------------- dispatch in the quantizer's store
 
 def run_dispatch(fq, X, token_rows, R, fmt="e4m3"):
-    Xq = torch.full((R, X.shape[1]), 0x7F, dtype=torch.uint8, device="cuda")
-    s = torch.full((R,), float("nan"), dtype=torch.float32, device="cuda")
+    # guard-banded outputs: a token row dispatched past the last grouped row
+    # (or a scale written past the scale array) changes the guard bytes
+    g = Guards()
+    Xq = g((R, X.shape[1]), torch.uint8, 0x7F, "Xq")
+    s = g((R,), torch.float32, float("nan"), "s_x")
     fq.quantize_rows_dispatch(X.cuda(), torch.from_numpy(token_rows).cuda(), R, out=(Xq, s), fmt=fmt)
-    torch.cuda.synchronize()
+    g.check("dispatch")
     return to_np(Xq), to_np(s)
 
 
@@ -161,12 +155,12 @@ def test_dispatch_then_grouped_linear_equals_gather(fq):
 
 
 def test_dispatch_moe_tokens(fq):
+    # every grouped row of the full-size dispatch, bit for bit
     m = wl.moe()
     row_token = np.asarray(m.token_of_row, dtype=np.int32)
     T = m.X.shape[0]
     got_q, got_s = run_dispatch(fq, m.X, wl.token_rows(row_token, T), len(row_token))
-    rows = sample_rows(len(row_token), 512, seed=14)
-    ref_q, ref_s = quant_rows(m.X.numpy()[row_token[rows]])
-    assert np.array_equal(got_q[rows], ref_q)
-    assert np.array_equal(got_s[rows].view(np.uint32), ref_s.view(np.uint32))
+    ref_q, ref_s = quant_rows(m.X.numpy())
+    assert np.array_equal(got_q, ref_q[row_token])
+    assert np.array_equal(got_s.view(np.uint32), ref_s[row_token].view(np.uint32))
     assert_no_device_error()

@@ -2,7 +2,11 @@
 
 Rows arrive grouped by expert (FP16 top-2 router and permutation are part of
 the seeded input synthesis); offsets live on the device.  The oracle computes
-every checked row with its expert's quantized weights and scales.
+every row with its expert's quantized weights and scales, and every row of
+every output is compared, the full-size 16384-row up and down projections
+included.  All device outputs sit inside guard-banded buffers (a seeded byte
+pattern on each side, checked after the call), so a masked store at an expert
+boundary that runs past the last row of the output is caught.
 """
 import numpy as np
 import pytest
@@ -11,7 +15,7 @@ import torch
 from oracle import linear_ref, moe_ref, quant_rows
 from fp8_quantized_generative_b200 import workloads as wl
 
-from parity import assert_close_f16, assert_no_device_error, sample_rows, to_np
+from parity import Guards, assert_close_f16, assert_no_device_error, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -24,12 +28,22 @@ def fq():
 
 
 def run_gpu(fq, Xg, offsets, W):
-    Wq, s_w = fq.quantize_weight_per_channel(W.cuda())
-    Xq, s_x = fq.quantize_rows_dynamic(Xg.cuda())
+    g = Guards()
+    E, N, K = W.shape
+    R = Xg.shape[0]
+    Wq = g((E, N, K), torch.uint8, 0xFF, "Wq")
+    s_w = g((E, N), torch.float32, float("nan"), "s_w")
+    fq.quantize_weight_per_channel(W.cuda(), out=(Wq, s_w))
+    Xq = g((R, K), torch.uint8, 0xFF, "Xq")
+    s_x = g((R,), torch.float32, float("nan"), "s_x")
+    fq.quantize_rows_dynamic(Xg.cuda(), out=(Xq, s_x))
     off = torch.from_numpy(np.asarray(offsets, dtype=np.int32)).cuda()
-    Y = torch.full((Xg.shape[0], W.shape[1]), float("nan"), dtype=torch.float16, device="cuda")
+    # NaN-filled, guard-banded output: rows written past an expert group's end
+    # land in a neighbour's rows (caught by the compare) or past the buffer
+    # (caught by the guard bytes)
+    Y = g((R, N), torch.float16, float("nan"), "Y")
     fq.moe_grouped_linear(Xq, s_x, off, Wq, s_w, out=Y)
-    torch.cuda.synchronize()
+    g.check(f"moe R={R} E={E} N={N} K={K}")
     return Y
 
 
@@ -112,10 +126,11 @@ def moe_case():
 
 
 def test_moe_up_full(fq, family, moe_case):
+    # every grouped row of the full-size up projection against the oracle
     m = moe_case
     Y = run_gpu(fq, m.X_perm, m.offsets, m.W_up)
-    rows = sample_rows(m.X_perm.shape[0], 256, seed=4)
-    assert_close_f16(to_np(Y)[rows], oracle_rows(m.X_perm, m.offsets, m.W_up, rows), "moe up")
+    R = m.X_perm.shape[0]
+    assert_close_f16(to_np(Y), oracle_rows(m.X_perm, m.offsets, m.W_up, np.arange(R)), "moe up")
     assert_no_device_error()
 
 
@@ -124,6 +139,5 @@ def test_moe_down_full(fq, family, moe_case):
     m = moe_case
     Xd = wl.random_f16((m.X_perm.shape[0], wl.MOE_F), seed=303)
     Y = run_gpu(fq, Xd, m.offsets, m.W_down)
-    rows = sample_rows(Xd.shape[0], 256, seed=5)
-    assert_close_f16(to_np(Y)[rows], oracle_rows(Xd, m.offsets, m.W_down, rows), "moe down")
+    assert_close_f16(to_np(Y), oracle_rows(Xd, m.offsets, m.W_down, np.arange(Xd.shape[0])), "moe down")
     assert_no_device_error()

@@ -5,7 +5,7 @@ warps quantize the fp16 rows while its tensor cores start on the row blocks
 already published.
 
 * the codes and scales it leaves in the workspace are bit-exact against
-  oracle.quant_rows (every row, or sampled rows at the QKV size);
+  oracle.quant_rows (every row, the full QKV size included);
 * Y is within the path's tolerance of oracle.linear_ref, and bitwise equal to
   the two-launch path (same tiles, same accumulation order);
 * the sync words are zero again after every call, so calls repeat (with the
@@ -18,7 +18,7 @@ import torch
 from oracle import linear_ref, quant_rows
 from fp8_quantized_generative_b200 import workloads as wl
 
-from parity import assert_close_f16, assert_no_device_error, sample_rows, to_np
+from parity import Guards, assert_close_f16, assert_no_device_error, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -34,10 +34,14 @@ def run(fq, X, W, ws=None):
     Wq, s_w = fq.quantize_weight_per_channel(W.cuda())
     Xd = X.cuda()
     M, K = X.shape
-    ws = ws if ws is not None else fq.overlap_workspace(M, K, "cuda")
-    Y = torch.full((M, W.shape[0]), float("nan"), dtype=torch.float16, device="cuda")
+    g = Guards()
+    if ws is None:
+        # guard-banded workspace: codes, scales and sync words
+        ws = (g((M, K), torch.uint8, 0xFF, "Xq_ws"), g((M,), torch.float32, float("nan"), "s_x_ws"),
+              g((int(fq._lib.fp8q_overlap_sync_words(M)),), torch.int32, 0, "sync"))
+    Y = g((M, W.shape[0]), torch.float16, float("nan"), "Y")
     fq.quantized_linear_overlapped(Xd, Wq, s_w, workspace=ws, out=Y)
-    torch.cuda.synchronize()
+    g.check(f"overlapped {M}x{W.shape[0]}x{K}")
     return Y, ws, (Xd, Wq, s_w)
 
 
@@ -109,12 +113,12 @@ def test_tile_widths(fq, bn):
 
 
 def test_qkv_projection(fq):
+    # the full QKV projection: every code, scale and output element
     lin = wl.qkv()
     Y, (Xq, s_x, _), _ = run(fq, lin.X, lin.W)
-    rows = sample_rows(lin.X.shape[0], 64, seed=15)
-    ref_q, ref_s = quant_rows(lin.X.numpy()[rows])
-    assert np.array_equal(to_np(Xq)[rows], ref_q)
-    assert np.array_equal(to_np(s_x)[rows].view(np.uint32), ref_s.view(np.uint32))
+    ref_q, ref_s = quant_rows(lin.X.numpy())
+    assert np.array_equal(to_np(Xq), ref_q)
+    assert np.array_equal(to_np(s_x).view(np.uint32), ref_s.view(np.uint32))
     rwq, rsw = quant_rows(lin.W.numpy())
-    assert_close_f16(to_np(Y)[rows], linear_ref(ref_q, ref_s, rwq, rsw), "overlapped qkv")
+    assert_close_f16(to_np(Y), linear_ref(ref_q, ref_s, rwq, rsw), "overlapped qkv")
     assert_no_device_error()

@@ -1,7 +1,9 @@
 """GPU parity of the per-row E4M3 quantizer and the device cast: bit-exact.
 
 Codes and scales from libfp8q are compared byte for byte with the CPU oracle
-(oracle.quant_rows / oracle.e4m3_encode) on the same seeded inputs.
+(oracle.quant_rows / oracle.e4m3_encode) on the same seeded inputs: every row
+of every matrix, the full-size ones included, with guard-banded outputs.  The
+device cast is swept over all 2^32 fp32 bit patterns (test_zy_cast_sweep.py).
 """
 import numpy as np
 import pytest
@@ -10,7 +12,7 @@ import torch
 from oracle import e4m3_encode, quant_rows
 from fp8_quantized_generative_b200 import workloads as wl
 
-from parity import assert_no_device_error, sample_rows, to_np
+from parity import Guards, assert_no_device_error, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -22,17 +24,18 @@ def fq():
     return m
 
 
-def _check_rows(fq, X, rows=None, what=""):
+def _check_rows(fq, X, what=""):
     Xd = X.cuda()
-    # sentinel-filled outputs: unwritten codes or scales fail the comparison
-    Xq = torch.full(X.shape, 0x7F, dtype=torch.uint8, device="cuda")
-    s = torch.full((X.shape[0],), float("nan"), dtype=torch.float32, device="cuda")
+    # sentinel-filled, guard-banded outputs: unwritten codes or scales fail
+    # the comparison, writes past either end fail the guard check
+    g = Guards()
+    Xq = g(X.shape, torch.uint8, 0x7F, "Xq")
+    s = g((X.shape[0],), torch.float32, float("nan"), "s")
     fq.quantize_rows_dynamic(Xd, out=(Xq, s))
-    torch.cuda.synchronize()
-    idx = np.arange(X.shape[0]) if rows is None else rows
-    ref_q, ref_s = quant_rows(X.numpy()[idx])
-    got_q = to_np(Xq)[idx]
-    got_s = to_np(s)[idx]
+    g.check(what)
+    ref_q, ref_s = quant_rows(X.numpy())
+    got_q = to_np(Xq)
+    got_s = to_np(s)
     if not np.array_equal(got_q, ref_q):
         bad = np.argwhere(got_q != ref_q)[0]
         raise AssertionError(f"{what}: code mismatch at {tuple(bad)}: gpu 0x{got_q[tuple(bad)]:02x} "
@@ -67,16 +70,16 @@ def test_edge_rows(fq):
 
 
 def test_full_size_activations(fq):
+    # every row of every full-size activation and weight matrix, bit for bit
     lin = wl.qkv()
     _check_rows(fq, lin.X, what="qkv X")
     _check_rows(fq, lin.W, what="qkv W")
     up, down = wl.ffn()
-    _check_rows(fq, up.X, rows=sample_rows(up.X.shape[0], 256, 1), what="ffn_up X")
-    _check_rows(fq, down.X, rows=sample_rows(down.X.shape[0], 128, 2), what="ffn_down X")
+    _check_rows(fq, up.X, what="ffn_up X")
+    _check_rows(fq, down.X, what="ffn_down X")
     _check_rows(fq, down.W, what="ffn_down W")
     for m in (1, 8, 128, 16384):
-        X = wl.sweep_x(m)
-        _check_rows(fq, X, rows=sample_rows(m, 256, m), what=f"sweep X m={m}")
+        _check_rows(fq, wl.sweep_x(m), what=f"sweep X m={m}")
 
 
 def test_moe_weights_per_channel(fq):
@@ -85,10 +88,10 @@ def test_moe_weights_per_channel(fq):
     Wq, s = fq.quantize_weight_per_channel(Wd)
     torch.cuda.synchronize()
     assert Wq.shape == m.W_up.shape and s.shape == m.W_up.shape[:2]
-    for e in (0, 17, 63):
-        ref_q, ref_s = quant_rows(m.W_up[e].numpy())
-        np.testing.assert_array_equal(to_np(Wq[e]), ref_q)
-        np.testing.assert_array_equal(to_np(s[e]).view(np.uint32), ref_s.view(np.uint32))
+    E, N, K = m.W_up.shape
+    ref_q, ref_s = quant_rows(m.W_up.reshape(E * N, K).numpy())
+    np.testing.assert_array_equal(to_np(Wq).reshape(E * N, K), ref_q)
+    np.testing.assert_array_equal(to_np(s).reshape(E * N).view(np.uint32), ref_s.view(np.uint32))
     assert_no_device_error()
 
 

@@ -167,6 +167,7 @@ struct Knobs {
   int bn = 0;
   int ksplit = 0; // split-K cluster size, 0 = automatic
   int half_tiles = 1; // FP8Q_HALF_TILES: 0 = CTA-pair grouped kernel uses only M = 256 tiles
+  int stage_k = 256;  // FP8Q_STAGE_K: K bytes per stage of the dense pair kernel (128 or 256)
 };
 Knobs& knobs() {
   static Knobs k = []() {
@@ -179,6 +180,7 @@ Knobs& knobs() {
     if (const char* k = std::getenv("FP8Q_KSPLIT")) r.ksplit = std::atoi(k);
     if (const char* b = std::getenv("FP8Q_BN")) r.bn = std::atoi(b);
     if (const char* h = std::getenv("FP8Q_HALF_TILES")) r.half_tiles = h[0] == '0' ? 0 : 1;
+    if (const char* v = std::getenv("FP8Q_STAGE_K")) r.stage_k = std::atoi(v) == 128 ? 128 : 256;
     return r;
   }();
   return k;
@@ -264,16 +266,16 @@ int l2_prefetch_enabled() {
 }
 
 // Per-device cache of how many 2-CTA clusters of a pair kernel fit at once.
-template <int BN, int STAGES, bool kGrouped>
+template <int BN, int STAGES, bool kGrouped, int SK = kBK>
 int max_pair_clusters(int dev) {
   static int cache[kMaxDevices] = {0};
   static std::mutex mu;
   std::lock_guard<std::mutex> g(mu);
   if (cache[dev] > 0) return cache[dev];
-  using L = PairLayout<BN, STAGES>;
-  auto kernel = fp8_gemm_pair_kernel<BN, STAGES, kGrouped>;
+  using L = PairLayout<BN, STAGES, SK>;
+  auto kernel = fp8_gemm_pair_kernel<BN, STAGES, kGrouped, false, SK>;
   const size_t smem = L::smem_bytes(kGrouped ? kMaxExperts : 0);
-  if (ensure_smem<fp8_gemm_pair_kernel<BN, STAGES, kGrouped>>(smem, dev) != cudaSuccess) {
+  if (ensure_smem<fp8_gemm_pair_kernel<BN, STAGES, kGrouped, false, SK>>(smem, dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return 0;
   }
@@ -328,11 +330,11 @@ TailSplit tail_split(int64_t full_tiles, int clusters, int bn) {
 // Launch a pair kernel.  Dense: A = Xq [rows, K], B = Wq [N, K].  Grouped:
 // B = Wq [E*N, K] and the schedule comes from the device offsets;
 // `tiles_upper_bound` caps the grid when the tile count is unknown on the host.
-template <int BN, int STAGES, bool kGrouped, bool kQuantA = false>
+template <int BN, int STAGES, bool kGrouped, bool kQuantA = false, int SK = kBK>
 fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, int64_t b_rows, const GemmParams& p0, int dev,
                         cudaStream_t st, int64_t tiles_upper_bound = 0) {
-  using L = PairLayout<BN, STAGES>;
-  const int clusters = max_pair_clusters<BN, STAGES, kGrouped>(dev);
+  using L = PairLayout<BN, STAGES, SK>;
+  const int clusters = max_pair_clusters<BN, STAGES, kGrouped, SK>(dev);
   if (clusters < 1) {
     g_last_error = "no 2-CTA cluster of the pair GEMM fits on this device";
     return FP8Q_ERR_UNSUPPORTED;
@@ -367,8 +369,8 @@ fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, int64_t b_rows, cons
   if (s != FP8Q_OK) return s;
   s = make_output_map(&ty, p.Y, p.rows, p.N);
   if (s != FP8Q_OK) return s;
-  auto kernel = fp8_gemm_pair_kernel<BN, STAGES, kGrouped, kQuantA>;
-  cudaError_t e = ensure_smem<fp8_gemm_pair_kernel<BN, STAGES, kGrouped, kQuantA>>(
+  auto kernel = fp8_gemm_pair_kernel<BN, STAGES, kGrouped, kQuantA, SK>;
+  cudaError_t e = ensure_smem<fp8_gemm_pair_kernel<BN, STAGES, kGrouped, kQuantA, SK>>(
       L::smem_bytes(kGrouped ? kMaxExperts : 0), dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair)");
   const int pairs = static_cast<int>(tiles < clusters ? (tiles < 1 ? 1 : tiles) : clusters);
@@ -522,6 +524,16 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
   if (pair) {
     const int clusters = max_pair_clusters<256, 6, false>(dev);
     int bn = kn.bn ? kn.bn : choose_pair_bn(p.rows, p.N, clusters > 0 ? clusters : sms / 2);
+    // Two 128-byte K boxes per stage (measured 3-10% faster on B200 than one:
+    // the MMA-issuing thread's per-stage work is spread over eight MMAs).
+    if (kn.stage_k == 256) {
+      switch (bn) {
+        case 128: return launch_pair<128, 4, false, false, 256>(Xq, Wq, p.N, q, dev, st);
+        case 192: return launch_pair<192, 3, false, false, 256>(Xq, Wq, p.N, q, dev, st);
+        case 512: return launch_pair<512, 4, false>(Xq, Wq, p.N, q, dev, st);
+        default: return launch_pair<256, 3, false, false, 256>(Xq, Wq, p.N, q, dev, st);
+      }
+    }
     switch (bn) {
       case 128: return launch_pair<128, 8, false>(Xq, Wq, p.N, q, dev, st);
       case 192: return launch_pair<192, 6, false>(Xq, Wq, p.N, q, dev, st);
@@ -799,10 +811,18 @@ fp8q_status fp8q_quantized_linear_overlapped(const void* X_f16, const uint8_t* W
   p.n_fastest = raster == 1 ? 0 : 1;
   const int clusters = max_pair_clusters<256, 6, false>(dev);
   const int bn = kn.bn ? kn.bn : choose_pair_bn(M, N, clusters > 0 ? clusters : sms / 2);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (kn.stage_k == 256) {
+    switch (bn) {
+      case 128: return launch_pair<128, 4, false, true, 256>(Xq_ws, Wq, N, p, dev, st);
+      case 192: return launch_pair<192, 3, false, true, 256>(Xq_ws, Wq, N, p, dev, st);
+      default: return launch_pair<256, 3, false, true, 256>(Xq_ws, Wq, N, p, dev, st);
+    }
+  }
   switch (bn) {
-    case 128: return launch_pair<128, 8, false, true>(Xq_ws, Wq, N, p, dev, static_cast<cudaStream_t>(stream));
-    case 192: return launch_pair<192, 6, false, true>(Xq_ws, Wq, N, p, dev, static_cast<cudaStream_t>(stream));
-    default: return launch_pair<256, 6, false, true>(Xq_ws, Wq, N, p, dev, static_cast<cudaStream_t>(stream));
+    case 128: return launch_pair<128, 8, false, true>(Xq_ws, Wq, N, p, dev, st);
+    case 192: return launch_pair<192, 6, false, true>(Xq_ws, Wq, N, p, dev, st);
+    default: return launch_pair<256, 6, false, true>(Xq_ws, Wq, N, p, dev, st);
   }
 }
 

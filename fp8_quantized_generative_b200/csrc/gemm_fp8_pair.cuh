@@ -30,11 +30,17 @@
 
 namespace fp8q {
 
-template <int BN, int STAGES>
+// SK: K bytes per pipeline stage, kBK (one 128-byte swizzle box per operand)
+// or 2 * kBK (two boxes side by side: eight MMAs per barrier round trip
+// instead of four, halving the issuing thread's per-MMA bookkeeping).
+template <int BN, int STAGES, int SK = kBK>
 struct PairLayout {
-  static constexpr int kABytes = kBM * kBK;            // own 128 rows of A
+  static constexpr int kBoxes = SK / kBK;              // 128-byte K boxes per operand per stage
+  static constexpr int kABox = kBM * kBK;
+  static constexpr int kABytes = kBM * SK;             // own 128 rows of A
   static constexpr int kBRows = BN / 2;                // own half of the B rows
-  static constexpr int kBBytes = kBRows * kBK;
+  static constexpr int kBBox = kBRows * kBK;
+  static constexpr int kBBytes = kBRows * SK;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kNumBars = 2 * STAGES + 5;      // full, empty, tfull[2], tempty[2], drain
   static constexpr int kTmemCols = 512;
@@ -115,12 +121,13 @@ __device__ __forceinline__ PairTile pair_tile(int t, const GemmParams& p, int nu
   return r;
 }
 
-template <int BN, int STAGES, bool kGrouped, bool kQuantA = false>
+template <int BN, int STAGES, bool kGrouped, bool kQuantA = false, int SK = kBK>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAh,
                          const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBt,
                          const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
-  using L = PairLayout<BN, STAGES>;
+  using L = PairLayout<BN, STAGES, SK>;
+  static_assert(SK == kBK || (SK == 2 * kBK && BN <= 256), "stage K: one box, or two for tiles up to 256 wide");
   static_assert(BN % 64 == 0 && BN >= 64 && (BN <= 256 || BN == 512) && (BN / 2) % 8 == 0, "BN");
   static_assert(L::kNAcc * BN <= L::kTmemCols, "accumulators must fit in TMEM");
   static_assert(!(kQuantA && kGrouped), "in-kernel quantization is the dense form");
@@ -155,7 +162,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int npairs = static_cast<int>(gridDim.x >> 1);
   const int num_m = (p.rows + 2 * kBM - 1) / (2 * kBM);
   const int num_n = (p.N + BN - 1) / BN;
-  const int num_kb = (p.K + kBK - 1) / kBK;
+  const int num_kb = (p.K + SK - 1) / SK;   // pipeline stages of SK bytes of K
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -229,8 +236,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int h = 0; h < pt.bn / 256; ++h)
           tma_load_2d_pair(dst + h * 128 * kBK, &tmB, bar, kx, pt.b_row0 + 256 * h + static_cast<int>(rank) * 128);
       } else {
-        tma_load_2d_pair(dst, pt.tail ? &tmBt : &tmB, bar, kx, pt.b_row0 + static_cast<int>(rank) * (pt.bn / 2));
+#pragma unroll
+        for (int j = 0; j < L::kBoxes; ++j)
+          tma_load_2d_pair(dst + j * L::kBBox, pt.tail ? &tmBt : &tmB, bar, kx + j * kBK,
+                           pt.b_row0 + static_cast<int>(rank) * (pt.bn / 2));
       }
+    };
+    // This CTA's A rows for one stage: kBoxes boxes of 128 bytes of K.
+    auto load_a = [&](uint8_t* dst, const CUtensorMap* tm, uint32_t bar, int kx, int row) {
+#pragma unroll
+      for (int j = 0; j < L::kBoxes; ++j) tma_load_2d_pair(dst + j * L::kABox, tm, bar, kx + j * kBK, row);
     };
     // The weights do not depend on the kernel launched before this one
     // (programmatic dependent launch): request the first ring pass of the
@@ -239,12 +254,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int pre = 0;
     if (lane == 0 && !kGrouped && pair < total) {
       const PairTile pt = pair_tile<BN, kGrouped>(pair, p, num_m, num_n, tile_prefix, offs);
-      const uint32_t bytes = 2u * static_cast<uint32_t>(L::kABytes + (pt.bn / 2) * kBK);
+      const uint32_t bytes = 2u * static_cast<uint32_t>(L::kABytes + (pt.bn / 2) * SK);
       pre = num_kb < STAGES ? num_kb : STAGES;
       for (int i = 0; i < pre; ++i) {
         const uint32_t full_leader = mapa_shared(smem_u32(&full[i]), 0);
         if (leader) mbar_arrive_expect_tx(&full[i], bytes);
-        load_b(pt, sB + i * L::kBBytes, full_leader, i * kBK);
+        load_b(pt, sB + i * L::kBBytes, full_leader, i * SK);
       }
     }
     __syncwarp();
@@ -262,7 +277,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int a_rows = pt.half ? kBM / 2 : kBM;
         const int a_row = pt.a_row0 + static_cast<int>(rank) * a_rows;
         const CUtensorMap* tma_a = pt.half ? &tmAh : &tmA;
-        const uint32_t bytes = 2u * static_cast<uint32_t>(a_rows * kBK + (pt.bn / 2) * kBK);
+        const uint32_t bytes = 2u * static_cast<uint32_t>(a_rows * SK + (pt.bn / 2) * SK);
         if (kQuantA && !ready.wait(p, a_row, true)) {   // this CTA's 128 rows quantized
           ok = false;
           break;
@@ -271,7 +286,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (pre > 0) {
             // stage kb of the first pass: weights already requested
             const uint32_t full_leader = mapa_shared(smem_u32(&full[s]), 0);
-            tma_load_2d_pair(sA + s * L::kABytes, &tmA, full_leader, kb * kBK, a_row);
+            load_a(sA + s * L::kABytes, &tmA, full_leader, kb * SK, a_row);
             --pre;
             if (++s == STAGES) {
               s = 0;
@@ -285,8 +300,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint32_t full_leader = mapa_shared(smem_u32(&full[s]), 0);
           if (leader) mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_2d_pair(sA + s * L::kABytes, tma_a, full_leader, kb * kBK, a_row);
-          load_b(pt, sB + s * L::kBBytes, full_leader, kb * kBK);
+          load_a(sA + s * L::kABytes, tma_a, full_leader, kb * SK, a_row);
+          load_b(pt, sB + s * L::kBBytes, full_leader, kb * SK);
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;
@@ -313,6 +328,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int s = 0, acc = 0;
       uint32_t ph = 0, acc_ph = 0;
       bool issued = false, ok = true;
+      // Addresses and descriptors of stage 0; stage s adds s times the stage
+      // size (the descriptor's start-address field counts 16-byte units).
+      // Keeping this loop's instruction stream short matters: the issuing
+      // thread's scalar work between tensor-core instructions is slow
+      // while MMAs are in flight.
+      const uint32_t full_a = smem_u32(full), empty_a = smem_u32(empty);
+      const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(sA)), bdesc0 = sw128_kmajor_desc(smem_u32(sB));
       for (int t = pair; t < total && ok; t += npairs) {
         if (!mbar_wait(&tempty[acc], acc_ph ^ 1u, abort_flag)) {
           ok = false;
@@ -326,21 +348,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           idesc = idesc_e4m3_f32(kBM, BN) | kAFmt;
         const int halves = kWide ? pair_tile<BN, kGrouped>(t, p, num_m, num_n, tile_prefix, offs).bn / 256 : 1;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[s], ph, abort_flag)) {
+          if (!mbar_wait_addr(full_a + 8u * s, ph, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t a0 = sw128_kmajor_desc(smem_u32(sA + s * L::kABytes));
-          const uint64_t b0 = sw128_kmajor_desc(smem_u32(sB + s * L::kBBytes));
+          const uint64_t a0 = adesc0 + static_cast<uint64_t>(s * (L::kABytes >> 4));
+          const uint64_t b0 = bdesc0 + static_cast<uint64_t>(s * (L::kBBytes >> 4));
 #pragma unroll
-          for (int k = 0; k < kBK / kUmmaK; ++k)
+          for (int k = 0; k < SK / kUmmaK; ++k) {
+            // box k / 4 of the stage, 32-byte step k % 4 inside its swizzle row
+            const int box = k / (kBK / kUmmaK), kin = k % (kBK / kUmmaK);
             for (int h = 0; h < halves; ++h)   // wide: N = 256 halves at TMEM columns 256h
-              mma_f8f6f4_pair(d + static_cast<uint32_t>(256 * h), a0 + static_cast<uint64_t>(k * kUmmaK / 16),
-                              b0 + static_cast<uint64_t>(h * 128 * kBK / 16 + k * kUmmaK / 16), idesc,
-                              (kb | k) != 0 ? 1u : 0u);
+              mma_f8f6f4_pair(d + static_cast<uint32_t>(256 * h),
+                              a0 + static_cast<uint64_t>(box * (L::kABox >> 4) + kin * kUmmaK / 16),
+                              b0 + static_cast<uint64_t>(box * (L::kBBox >> 4) + h * 128 * kBK / 16 + kin * kUmmaK / 16),
+                              idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           issued = true;
-          mma_commit_pair_mc(&empty[s], 0x3);
+          mma_commit_pair_mc_addr(empty_a + 8u * s, 0x3);
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;

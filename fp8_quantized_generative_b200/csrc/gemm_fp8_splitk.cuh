@@ -62,6 +62,59 @@ struct SplitKLayout {
   }
 };
 
+// The owner's share of the split-K reduction: the S partial slices of its
+// kBM / S weight rows (its own slice in the send buffer, the peers' in the
+// receive buffer) summed in rank order 0..S-1, scaled and stored as fp16.
+// Each of the 128 epilogue threads takes blocks of 4 token rows x 8 weight
+// rows: eight 16-byte shared loads per slice, one 16-byte global store per
+// token row (the 8 outputs are consecutive columns of Y).
+template <int S, typename L>
+__device__ __forceinline__ void splitk_reduce_store(const GemmParams& p, const float* send, const float* recv,
+                                                    const float* sc_w, const float* sc_x, int n0, int rank, int et) {
+  constexpr int SL = kBM / S;
+  constexpr int NB = SL / 8;                       // 8-row blocks per owner
+  const int m4n = (p.rows + 3) >> 2;
+  const int items = m4n * NB;
+  for (int idx = et; idx < items; idx += 128) {
+    const int nl0 = (idx % NB) * 8;
+    const int m = (idx / NB) * 4;
+    const int n = n0 + rank * SL + nl0;
+    if (n >= p.N) continue;                        // N % 8 == 0: a block is all in or all out
+    float acc[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+#pragma unroll
+    for (int s2 = 0; s2 < S; ++s2) {
+      const float* base =
+          (s2 == rank ? send + (rank * SL + nl0) * L::kPitch : recv + (s2 * SL + nl0) * L::kPitch) + m;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 v = *reinterpret_cast<const float4*>(base + j * L::kPitch);
+        acc[j][0] = __fadd_rn(acc[j][0], v.x);
+        acc[j][1] = __fadd_rn(acc[j][1], v.y);
+        acc[j][2] = __fadd_rn(acc[j][2], v.z);
+        acc[j][3] = __fadd_rn(acc[j][3], v.w);
+      }
+    }
+    float sw[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sw[j] = sc_w[nl0 + j];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (m + i >= p.rows) break;
+      const float sx = sc_x[m + i];
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        const __half2 h = __floats2half2_rn(__fmul_rn(__fmul_rn(acc[j][i], sx), sw[j]),
+                                            __fmul_rn(__fmul_rn(acc[j + 1][i], sx), sw[j + 1]));
+        w[j / 2] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      *reinterpret_cast<uint4*>(p.Y + static_cast<int64_t>(m + i) * p.N + n) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
 template <int MPAD, int STAGES, bool kFused>
 __global__ void __launch_bounds__(kSkThreads, 1)
     fp8_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -300,20 +353,25 @@ __global__ void __launch_bounds__(kSkThreads, 1)
               make_float4(have ? __uint_as_float(v[i]) : 0.f, have ? __uint_as_float(v[i + 1]) : 0.f,
                           have ? __uint_as_float(v[i + 2]) : 0.f, have ? __uint_as_float(v[i + 3]) : 0.f);
     } else {
-#pragma unroll 1
+      // 32 columns at a time, the TMEM load of chunk c+1 in flight while
+      // chunk c is written out.
+      const int nch = (mcols + 31) / 32;
+      uint32_t v[2][32];
+      if (have) tmem_ld_32x32b_x32(taddr, v[0]);
+#pragma unroll
       for (int c = 0; c < MPAD / 32; ++c) {
-        if (c * 32 >= mcols) break;
-        uint32_t v[32];
+        if (c >= nch) break;
         if (have) {
-          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(v[c & 1]);
+          if (c + 1 < nch) tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>((c + 1) * 32), v[(c + 1) & 1]);
         }
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
           if (c * 32 + i < mcols)
             *reinterpret_cast<float4*>(dst + c * 32 + i) =
-                make_float4(have ? __uint_as_float(v[i]) : 0.f, have ? __uint_as_float(v[i + 1]) : 0.f,
-                            have ? __uint_as_float(v[i + 2]) : 0.f, have ? __uint_as_float(v[i + 3]) : 0.f);
+                make_float4(have ? __uint_as_float(v[c & 1][i]) : 0.f, have ? __uint_as_float(v[c & 1][i + 1]) : 0.f,
+                            have ? __uint_as_float(v[c & 1][i + 2]) : 0.f,
+                            have ? __uint_as_float(v[c & 1][i + 3]) : 0.f);
       }
     }
     tc_fence_before();
@@ -331,28 +389,11 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       raise_error(0x10u);
       *abort_flag = 1;
     } else {
-      const int m4n = (p.rows + 3) >> 2;
-      const int items = SL * m4n;
-      for (int idx = et; idx < items; idx += 128) {
-        const int nl = idx % SL;
-        const int m = (idx / SL) * 4;
-        const int n = n0 + rank * SL + nl;
-        if (n >= p.N) continue;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s2 = 0; s2 < S; ++s2) {
-          const float* src = s2 == rank ? send + (rank * SL + nl) * L::kPitch : recv + (s2 * SL + nl) * L::kPitch;
-          const float4 v = *reinterpret_cast<const float4*>(src + m);
-          acc.x = __fadd_rn(acc.x, v.x);
-          acc.y = __fadd_rn(acc.y, v.y);
-          acc.z = __fadd_rn(acc.z, v.z);
-          acc.w = __fadd_rn(acc.w, v.w);
-        }
-        const float sw = sc_w[nl];
-        const float a[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (m + j < p.rows)
-            p.Y[static_cast<int64_t>(m + j) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(a[j], sc_x[m + j]), sw));
+      switch (S) {
+        case 1: splitk_reduce_store<1, L>(p, send, recv, sc_w, sc_x, n0, rank, et); break;
+        case 2: splitk_reduce_store<2, L>(p, send, recv, sc_w, sc_x, n0, rank, et); break;
+        case 4: splitk_reduce_store<4, L>(p, send, recv, sc_w, sc_x, n0, rank, et); break;
+        default: splitk_reduce_store<8, L>(p, send, recv, sc_w, sc_x, n0, rank, et); break;
       }
     }
   }

@@ -159,3 +159,27 @@ def test_splitk_variants(fq, ksplit, M, N, K):
         check(fq, X, W, what=f"splitk S={ksplit} {M}x{N}x{K}")
     finally:
         fq.set_gemm_tuning(0, 0, 0)
+
+
+def test_one_box_stages_path_in_a_subprocess():
+    # The dense CTA-pair kernel runs 256-byte K stages by default; the
+    # one-box (128-byte) stage form stays selectable (FP8Q_STAGE_K=128, read
+    # once per process), so it is checked against the oracle in a process of
+    # its own, on ragged and multi-round shapes.
+    import os
+    import subprocess
+    import sys
+    code = r'''
+import sys, torch
+sys.path.insert(0, "tests")
+from test_gpu_linear import check
+import fp8_quantized_generative_b200 as fq
+from fp8_quantized_generative_b200 import workloads as wl
+for M, N, K in [(300, 520, 272), (1024, 6144, 2048), (257, 1000, 1040)]:
+    check(fq, wl.random_f16((M, K), seed=M + K), wl.random_f16((N, K), seed=N, std=0.02), what=f"{M}x{N}x{K}")
+print("ok")
+'''
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, FP8Q_STAGE_K="128")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]

@@ -141,13 +141,13 @@ def linear(Xq: torch.Tensor, s_x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Ten
     return Y
 
 
-FUSED_MAX_ROWS = 16
+FUSED_MAX_ROWS = 64
 
 
 def quantized_linear(X: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
                      out: torch.Tensor | None = None, fused: bool = False) -> torch.Tensor:
     """fp16 activations in, fp16 out: per-token quantization + FP8 linear +
-    dequantization.  fused=True runs one kernel (up to 16 rows, no workspace);
+    dequantization.  fused=True runs one kernel (up to 64 rows, no workspace);
     otherwise the two steps through a workspace allocated here."""
     _need(X, torch.float16, "X", 2)
     _need(Wq, torch.uint8, "Wq", 2)

@@ -151,8 +151,7 @@ fp8q_status make_output_map(CUtensorMap* m, const void* base, int64_t rows, int6
 }
 
 // ------------------------------------------------------------------ GEMM launch
-constexpr int kFusedMaxRows = 16;     // fused quantize + GEMM: token rows
-constexpr int kFusedMaxKBlocks = 32;  // ... and K blocks (of 128) per CTA
+constexpr int kFusedMaxRows = 64;     // fused quantize + GEMM: token rows
 constexpr int kBN = 256;        // single-CTA dense tiles (128 x 256)
 constexpr int kStages = 4;
 constexpr int kBNGrouped = 256; // MoE tiles (128 x 256); 128-wide tiles measured slower on B200
@@ -415,9 +414,9 @@ int max_splitk_clusters(int dev, int S) {
   static std::mutex mu;
   std::lock_guard<std::mutex> g(mu);
   if (cache[dev][S] != 0) return cache[dev][S];
-  using L = SplitKLayout<MPAD, STAGES>;
+  using L = SplitKLayout<MPAD, STAGES, kFused>;
   auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>;
-  const size_t max_smem = kFused ? L::fused_smem_bytes(kFusedMaxKBlocks) : L::kSmemBytes;
+  const size_t max_smem = kFused ? L::fused_smem_bytes(L::kFusedMaxKBlocks) : L::kSmemBytes;
   if (ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>>(max_smem, dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return -1;
@@ -465,7 +464,7 @@ int choose_ksplit(int dev, int n_tiles, int num_kb) {
 // otherwise A is Xq with scales s_x.
 template <int MPAD, int STAGES, bool kFused>
 fp8q_status launch_splitk(const uint8_t* Xq, const uint8_t* Wq, const GemmParams& p, int dev, cudaStream_t st) {
-  using L = SplitKLayout<MPAD, STAGES>;
+  using L = SplitKLayout<MPAD, STAGES, kFused>;
   CUtensorMap tw, tx;
   fp8q_status s = make_operand_map(&tw, Wq, p.N, p.K, kBM);
   if (s != FP8Q_OK) return s;
@@ -479,14 +478,14 @@ fp8q_status launch_splitk(const uint8_t* Xq, const uint8_t* Wq, const GemmParams
   const int num_kb = (p.K + kBK - 1) / kBK;
   const int S = knobs().ksplit ? knobs().ksplit : choose_ksplit<MPAD, STAGES, kFused>(dev, n_tiles, num_kb);
   const int nkb_max = (num_kb + S - 1) / S;
-  if (kFused && nkb_max > kFusedMaxKBlocks) {
+  if (kFused && nkb_max > L::kFusedMaxKBlocks) {
     g_last_error = "fused path: too many K blocks per CTA";
     return FP8Q_ERR_UNSUPPORTED;
   }
   const size_t smem = kFused ? L::fused_smem_bytes(nkb_max) : L::kSmemBytes;
   auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>;
   cudaError_t e = ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>>(
-      kFused ? L::fused_smem_bytes(kFusedMaxKBlocks) : L::kSmemBytes, dev);
+      kFused ? L::fused_smem_bytes(L::kFusedMaxKBlocks) : L::kSmemBytes, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(splitk)");
   e = launch_ex(kernel, dim3(n_tiles * S), dim3(kSkThreads), smem, st, S, true, tw, tx, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_splitk_kernel launch");
@@ -609,28 +608,28 @@ constexpr size_t kNoAllocCodeBytes = size_t(8) << 20;    // M * K codes
 constexpr size_t kNoAllocScaleCount = size_t(16) << 10;  // M scales
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocCodeBytes + kNoAllocScaleCount * 4];
 
-// Device address of the scratch array, resolved once per device with that
-// device current (host code cannot use the array's name as a device pointer).
+// Device address of the scratch array, looked up with that device current
+// (host code cannot use the array's name as a device pointer) and kept once
+// the lookup has succeeded; a failed lookup is not kept, so a later call
+// tries again.
 static fp8q_status noalloc_scratch(uint8_t** out) {
-  struct Slot {
-    std::once_flag once;
-    uint8_t* ptr = nullptr;
-    cudaError_t err = cudaSuccess;
-  };
-  static Slot slots[kMaxDevices];
+  static uint8_t* slots[kMaxDevices] = {};
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice, "device index");
-  Slot& sl = slots[dev];
-  std::call_once(sl.once, [&]() {
+  std::lock_guard<std::mutex> g(mu);
+  if (slots[dev] == nullptr) {
     void* p = nullptr;
-    sl.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    sl.ptr = static_cast<uint8_t*>(p);
-  });
-  if (sl.err != cudaSuccess || sl.ptr == nullptr)
-    return cuda_fail(sl.err != cudaSuccess ? sl.err : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
-  *out = sl.ptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
+    }
+    slots[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = slots[dev];
   return FP8Q_OK;
 }
 
@@ -742,11 +741,9 @@ fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const fl
   const bool have_ws = Xq_ws != nullptr || s_x_ws != nullptr;
   if (have_ws && (!aligned16(Xq_ws) || !aligned16(s_x_ws))) return invalid("workspace pointers must both be 16-byte aligned");
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // With a workspace: the two launches (on B200 the faster choice -- the
-  // quantizer's launch and the GEMM's weight prefetch overlap through
-  // programmatic dependent launch, while the fused kernel must read whole
-  // fp16 rows for their maxima before its first MMA).  Without one: the
-  // fused kernel, up to 16 rows.
+  // With a workspace: the two launches.  Without one: the fused kernel, up
+  // to 64 rows (the CTAs of a split-K cluster share the row maxima of their
+  // K slices, so no CTA reads whole fp16 rows).
   if (!have_ws && M <= kFusedMaxRows) {
     int dev = 0, sms = 0;
     const cudaError_t e = current_device_info(&dev, &sms);
@@ -761,7 +758,9 @@ fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const fl
     p.E = 1;
     p.tail_q = 1;
     p.l2_prefetch = l2_prefetch_enabled();
-    const fp8q_status s = launch_splitk<16, 5, true>(nullptr, Wq, p, dev, st);
+    const fp8q_status s = M <= 16 ? launch_splitk<16, 5, true>(nullptr, Wq, p, dev, st)
+                          : M <= 32 ? launch_splitk<32, 3, true>(nullptr, Wq, p, dev, st)
+                                    : launch_splitk<64, 3, true>(nullptr, Wq, p, dev, st);
     if (s != FP8Q_ERR_UNSUPPORTED) return s;   // else: too long a K slice, use the two-step path
   }
   if (!have_ws) return invalid("Xq_ws and s_x_ws are required for this shape (two-step path)");

@@ -134,7 +134,9 @@ __device__ __forceinline__ EpiScales<kMaxChunks> epilogue_scales(const EpiTile& 
                                                                  const EpiWarpView& w, int lane) {
   EpiScales<kMaxChunks> e;
   const int r = w.qrow0 + lane;
-  e.sx = r < t.row_end ? __ldg(p.s_x + act_row(p, r)) : 0.0f;
+  // With the quantization inside the GEMM (q_out set) s_x is still being
+  // written by this kernel: the caller reads it after its block's acquire.
+  e.sx = (p.q_out == nullptr && r < t.row_end) ? __ldg(p.s_x + act_row(p, r)) : 0.0f;
   e.rw = 0.0f;
   e.ctok = -1;
   if (p.comb_token != nullptr && r < t.row_end) {

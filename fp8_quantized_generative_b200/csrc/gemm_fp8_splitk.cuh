@@ -20,12 +20,14 @@
 //     slices locally in fixed rank order 0..S-1 (reproducible), applies the
 //     scales (staged in shared memory beforehand) and writes fp16 -- no
 //     global scratch memory;
-//   * fused variant (kFused, at most 16 token rows): the kernel takes the
-//     fp16 activations, and each CTA computes the per-row maxima and scales
-//     itself (the same fp32 steps as quant_rows.cuh) and writes the E4M3
-//     codes of its K slice straight into the 128-byte-swizzled K-major
-//     shared-memory layout the MMA reads -- quantize + GEMM + dequantize in
-//     one launch ("FP8量化在生成式推荐系统OneRec-V2中的优化实践" §2.3);
+//   * fused variant (kFused, at most 64 token rows): the kernel takes the
+//     fp16 activations; each CTA reads only its K slice of them, the row
+//     maxima of the slices are exchanged within the cluster (DSMEM bulk
+//     copies), and each CTA derives the per-row scales (the same fp32 steps
+//     as quant_rows.cuh) and writes the E4M3 codes of its K slice straight
+//     into the 128-byte-swizzled K-major shared-memory layout the MMA reads
+//     -- quantize + GEMM + dequantize in one launch
+//     ("FP8量化在生成式推荐系统OneRec-V2中的优化实践" §2.3);
 //   * the weight tiles do not depend on the kernel launched before this one,
 //     so the first STAGES of them are requested before the programmatic-
 //     dependent-launch wait: their DRAM latency overlaps that kernel's tail.
@@ -38,11 +40,15 @@ namespace fp8q {
 
 constexpr int kSkThreads = 192;   // producer, MMA, 4 epilogue warps
 
-template <int MPAD, int STAGES>
+// kFused: only the weight tiles travel through the ring (the activation
+// codes are made in shared memory), so a stage is a weight tile alone and the
+// CTA stays small enough for two to share an SM (the next kernel's CTAs can
+// then start and stream their weights while this one finishes).
+template <int MPAD, int STAGES, bool kFused = false>
 struct SplitKLayout {
   static constexpr int kWBytes = kBM * kBK;            // 128 weight rows x 128 K bytes
   static constexpr int kXBytes = MPAD * kBK;           // MPAD token rows
-  static constexpr int kStageBytes = kWBytes + kXBytes;
+  static constexpr int kStageBytes = kFused ? kWBytes : kWBytes + kXBytes;
   static constexpr int kRingBytes = STAGES * kStageBytes;
   // Partial rows of MPAD + 4 fp32 words (16-byte aligned rows; the +4 keeps
   // 8 consecutive rows of a 16-byte access on distinct bank groups).
@@ -50,16 +56,19 @@ struct SplitKLayout {
   static constexpr int kPartBytes = kBM * kPitch * 4;  // send buffer (in the ring) and receive buffer
   static_assert(kRingBytes >= kPartBytes, "the send buffer reuses the load ring");
   static constexpr int kScaleFloats = 128 + MPAD;      // owner's s_w slice + the token scales
-  static constexpr int kNumBars = 2 * STAGES + 4;      // full, empty, tfull, drain, recv, xready
+  static constexpr int kNumBars = 2 * STAGES + 5;      // full, empty, tfull, drain, recv, xready, pmax
   static constexpr int kTmemCols = MPAD < 32 ? 32 : MPAD;
   static constexpr int kBaseBytes = kRingBytes + kPartBytes + kScaleFloats * 4 + kNumBars * 8 + 32;
   static constexpr size_t kSmemBytes = 1024 + size_t(kBaseBytes);
   // Fused variant: 1024-aligned region after the base holding the E4M3 codes
-  // of the CTA's K blocks (MPAD x 128 bytes each) and the row statistics.
+  // of the CTA's K blocks (MPAD x 128 bytes each), then the partial row
+  // maxima of every CTA of the cluster (up to 8 x MPAD) and the row scales.
   static constexpr int kFusedOffset = (kBaseBytes + 1023) & ~1023;
   static size_t fused_smem_bytes(int nkb) {
-    return 1024 + size_t(kFusedOffset) + size_t(nkb) * kXBytes + 2 * MPAD * 4;
+    return 1024 + size_t(kFusedOffset) + size_t(nkb) * kXBytes + (8 + 1) * MPAD * 4;
   }
+  // Most K blocks per CTA the fused form takes (its codes stay in shared memory).
+  static constexpr int kFusedMaxKBlocks = MPAD <= 32 ? 32 : 16;
 };
 
 // The owner's share of the split-K reduction: the S partial slices of its
@@ -119,7 +128,7 @@ template <int MPAD, int STAGES, bool kFused>
 __global__ void __launch_bounds__(kSkThreads, 1)
     fp8_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                            const GemmParams p) {
-  using L = SplitKLayout<MPAD, STAGES>;
+  using L = SplitKLayout<MPAD, STAGES, kFused>;
   static_assert(MPAD % 16 == 0 && MPAD >= 16 && MPAD <= 128, "MPAD");
   // swap-AB: B = activations (E4M3, or E5M2 for the variant; the fused path is E4M3)
   const uint32_t kIdesc = idesc_e4m3_f32(kBM, MPAD) | idesc_b_fmt(kFused ? kFmtE4M3 : p.x_fmt);
@@ -140,6 +149,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   uint64_t* drain = bars + 2 * STAGES + 1;
   uint64_t* recv_bar = bars + 2 * STAGES + 2;
   uint64_t* xready = bars + 2 * STAGES + 3;   // fused: the CTA's activation codes are in place
+  uint64_t* pmax_bar = bars + 2 * STAGES + 4; // fused: the peers' partial row maxima have arrived
   uint8_t* fz_codes = smem + L::kFusedOffset;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -157,10 +167,14 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   const int SL = kBM / S;                          // weight rows owned by each CTA
   const int mcols = (p.rows + 3) & ~3;             // token rows carried, rounded to 4
   const uint32_t slice_bytes = static_cast<uint32_t>(SL * L::kPitch * 4);
-  float* fz_amax = reinterpret_cast<float*>(fz_codes + nkb * L::kXBytes);
-  float* fz_r = fz_amax + MPAD;
+  // The partial-maxima table sits at the same offset in every CTA of the
+  // cluster (peers copy into it by that offset): after the largest code
+  // region any rank has, not after this CTA's own.
+  const int nkb_max = (num_kb + S - 1) / S;
+  float* fz_pmax = reinterpret_cast<float*>(fz_codes + nkb_max * L::kXBytes);   // [S][MPAD]
+  float* fz_r = fz_pmax + 8 * MPAD;
   // Fused: only the weight tiles travel through the ring.
-  constexpr uint32_t kLoadBytes = kFused ? L::kWBytes : L::kStageBytes;
+  constexpr uint32_t kLoadBytes = L::kStageBytes;
 
   // Thread 0 is also the producer: it initializes the barriers and at once
   // requests the weight tiles of the first ring pass.  The weights do not
@@ -176,10 +190,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     mbar_init(drain, 1);
     mbar_init(recv_bar, 1);
     mbar_init(xready, 1);
+    mbar_init(pmax_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    // The S-1 peers' slices arrive as bulk copies counted on recv_bar.
+    // The S-1 peers' slices arrive as bulk copies counted on recv_bar (and,
+    // fused, their partial row maxima on pmax_bar).
     mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(S - 1) * slice_bytes);
+    if (kFused) mbar_arrive_expect_tx(pmax_bar, static_cast<uint32_t>(S - 1) * MPAD * 4);
     for (int i = 0; i < pre; ++i) {
       mbar_arrive_expect_tx(&full[i], kLoadBytes);
       tma_load_2d(sW + i * L::kWBytes, &tmW, &full[i], (kb0 + i) * kBK, n0);
@@ -284,48 +301,104 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       if (!kFused && et < p.rows) sc_x[et] = __ldg(p.s_x + et);
     }
     if (kFused) {
-      // Per-token dynamic quantization of the rows this CTA multiplies:
-      // row maxima over the whole K (warp w: rows w, w+4, ...), then the
-      // scales, then the codes of this CTA's K blocks in the swizzled
-      // layout of a 128-byte TMA box (row m at m*128, 16-byte chunk c at
-      // (c ^ (m & 7)) * 16).  Rows >= M and columns >= K are zero.
-      const int ew = warp - kEpiWarp0;
-      const int nvec = p.K >> 3;
-      for (int m = ew; m < p.rows; m += 4) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.x_f16 + static_cast<int64_t>(m) * p.K);
+      // Per-token dynamic quantization of the rows this CTA multiplies,
+      // shared by the S CTAs of the cluster, each of which reads only its
+      // own K slice of the fp16 rows: (1) the maxima of |x| over the slice
+      // go to slot [rank] of the partial-maxima
+      // table and are copied into the same slot of every peer (bulk
+      // shared-memory copies completing on the peer's pmax_bar); (2) each
+      // row's maximum is the max of its S partial maxima -- the same value,
+      // hence the same fp32 scale, on every CTA -- then r and s by the
+      // quantizer's steps; (3) the codes of this CTA's K blocks are written
+      // in the swizzled layout of a 128-byte TMA box (row m at m*128,
+      // 16-byte chunk c at (c ^ (m & 7)) * 16).  Rows >= M and columns >= K
+      // are zero.
+      // (1) T = 128 / MPAD consecutive threads per row, each taking every
+      // T-th 16-byte vector of the row's slice, eight loads in flight.
+      constexpr int T = 128 / MPAD;
+      const int v_lo = (kb0 * kBK) >> 3;
+      const int v_hi = (kb1 * kBK < p.K ? kb1 * kBK : p.K) >> 3;
+      float* own = fz_pmax + rank * MPAD;
+      {
+        const int m = et / T, sub = et % T;
         float a = 0.0f;
-        for (int j = lane; j < nvec; j += 32) a = absmax8(__ldg(src + j), a);
+        if (m < p.rows) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.x_f16 + static_cast<int64_t>(m) * p.K);
+          for (int j0 = v_lo + sub; j0 < v_hi; j0 += 8 * T) {
+            uint4 v[8];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        if (lane == 0) fz_amax[m] = a;
+            for (int u = 0; u < 8; ++u) v[u] = j0 + u * T < v_hi ? __ldg(src + j0 + u * T) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) a = absmax8(v[u], a);
+          }
+        }
+#pragma unroll
+        for (int o = T / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if (sub == 0 && m < p.rows) own[m] = a;
       }
+      fence_proxy_async_smem();
       named_barrier(1, 128);
+      bool got = true;
+      if (S > 1) {
+        // Every CTA of the cluster is running (arrived at set-up).  Only with
+        // peers: a launch without a cluster (S = 1) treats the cluster barrier
+        // as one over the whole CTA, whose MMA warp is waiting for these codes.
+        cluster_wait();
+        if (et < S && et != rank)
+          bulk_copy_to_cluster(mapa_shared(smem_u32(own), static_cast<uint32_t>(et)), own, MPAD * 4,
+                               mapa_shared(smem_u32(pmax_bar), static_cast<uint32_t>(et)));
+        got = mbar_wait(pmax_bar, 0, abort_flag);
+        if (!got) {
+          raise_error(0x10u);
+          *abort_flag = 1;
+        }
+      }
       if (et < p.rows) {
-        const RowScale rs = row_scale_from_amax(fz_amax[et]);
+        float a = 0.0f;
+        for (int s2 = 0; s2 < S; ++s2) a = fmaxf(a, fz_pmax[s2 * MPAD + et]);
+        const RowScale rs = row_scale_from_amax(a);
         fz_r[et] = rs.r;
         sc_x[et] = rs.s;
       }
       named_barrier(1, 128);
-      const int items = nkb * MPAD * 8;   // (k block, row, 16-byte chunk)
-      for (int it = et; it < items; it += 128) {
-        const int c = it & 7;
-        const int m = (it >> 3) % MPAD;
-        const int j = (it >> 3) / MPAD;
-        const int k = (kb0 + j) * kBK + c * 16;
-        uint4 out = make_uint4(0, 0, 0, 0);
-        if (m < p.rows && k < p.K) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.x_f16 + static_cast<int64_t>(m) * p.K + k);
-          const float r = fz_r[m];
-          const uint2 e0 = encode8(__ldg(src), r);
-          const uint2 e1 = encode8(__ldg(src + 1), r);
-          out = make_uint4(e0.x, e0.y, e1.x, e1.y);
+      // (3) items (k block, row, 16-byte chunk of codes), four per thread
+      // per round with all their loads issued first.
+      const int items = nkb * MPAD * 8;
+      for (int it0 = et; it0 < items; it0 += 4 * 128) {
+        uint4 x[4][2];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int it = it0 + u * 128;
+          const int m = (it >> 3) % MPAD;
+          const int k = (kb0 + (it >> 3) / MPAD) * kBK + (it & 7) * 16;
+          x[u][0] = x[u][1] = make_uint4(0, 0, 0, 0);
+          if (it < items && m < p.rows && k < p.K) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.x_f16 + static_cast<int64_t>(m) * p.K + k);
+            x[u][0] = __ldg(src);
+            x[u][1] = __ldg(src + 1);
+          }
         }
-        st_shared_v4(smem_u32(fz_codes + j * L::kXBytes + m * kBK) + static_cast<uint32_t>((c ^ (m & 7)) << 4), out.x,
-                     out.y, out.z, out.w);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int it = it0 + u * 128;
+          if (it >= items) break;
+          const int c = it & 7;
+          const int m = (it >> 3) % MPAD;
+          const int j = (it >> 3) / MPAD;
+          uint4 out = make_uint4(0, 0, 0, 0);
+          if (m < p.rows) {
+            const float r = fz_r[m];
+            const uint2 e0 = encode8(x[u][0], r);
+            const uint2 e1 = encode8(x[u][1], r);
+            out = make_uint4(e0.x, e0.y, e1.x, e1.y);
+          }
+          st_shared_v4(smem_u32(fz_codes + j * L::kXBytes + m * kBK) + static_cast<uint32_t>((c ^ (m & 7)) << 4),
+                       out.x, out.y, out.z, out.w);
+        }
       }
       fence_proxy_async_smem();
       named_barrier(1, 128);
-      if (et == 0) mbar_arrive(xready);
+      if (et == 0 && got) mbar_arrive(xready);
     }
     // Partial: TMEM lane = weight row n of the tile, column = token row m.
     const int q = warp & 3;
@@ -377,7 +450,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     tc_fence_before();
     fence_proxy_async_smem();
     named_barrier(1, 128);   // the four epilogue warps have written the whole send buffer
-    cluster_wait();          // every CTA of the cluster is running (arrived at set-up)
+    if (!kFused || S == 1) cluster_wait();   // every CTA of the cluster is running (fused: waited above)
     if (et < S && et != rank) {
       // ship owner et's rows to its receive slot [rank]
       const uint32_t peer_recv = mapa_shared(smem_u32(recv + rank * SL * L::kPitch), static_cast<uint32_t>(et));

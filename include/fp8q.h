@@ -44,6 +44,14 @@
  *     fp8q_device_error().
  *   - No call allocates device memory.  Results are bitwise reproducible from
  *     run to run (fixed reduction order everywhere).
+ *   - Kernels are chained with programmatic dependent launch: a kernel may
+ *     start while the one before it on the stream finishes, and waits for it
+ *     before touching its outputs.  The linear kernels treat the quantized
+ *     weights (Wq, s_w) as static and begin loading Wq before that wait, so
+ *     Wq must not be written by the work enqueued just before the call.  The
+ *     weight quantizers of this library (per channel, per tensor, block-wise)
+ *     let the next kernel start only once they have finished, so quantizing
+ *     the weights and then calling a linear on the same stream is safe.
  */
 #ifndef FP8Q_H_
 #define FP8Q_H_
@@ -119,11 +127,12 @@ fp8q_status fp8q_linear(const uint8_t* Xq, const float* s_x,
  *   fp8q_quantize_rows_dynamic followed by fp8q_linear.
  * With a workspace (Xq_ws [M,K] uint8 and s_x_ws [M] fp32, both non-NULL)
  * the call runs the two steps through it (the workspace then holds the codes
- * and scales); on B200 this is the faster choice.  With Xq_ws = s_x_ws = NULL
- * and up to 16 token rows (K up to 4096 x the split factor) it is one fused
- * kernel: each CTA computes the per-row scales and the E4M3 codes of its K
- * slice in shared memory, so no intermediate touches HBM.  NULL workspace
- * with a larger shape returns FP8Q_ERR_INVALID_ARG.
+ * and scales).  With Xq_ws = s_x_ws = NULL and up to 64 token rows (K up to
+ * 4096 x the split factor) it is one fused kernel: the CTAs of a split-K
+ * cluster each take the row maxima over their own K slice, exchange them,
+ * and write the E4M3 codes of their slice in shared memory, so no
+ * intermediate touches HBM.  NULL workspace with a larger shape returns
+ * FP8Q_ERR_INVALID_ARG.
  */
 fp8q_status fp8q_quantized_linear(const void* X_f16, const uint8_t* Wq, const float* s_w,
                                   int64_t M, int64_t N, int64_t K, void* Y_f16,
@@ -166,7 +175,8 @@ int64_t fp8q_overlap_sync_words(int64_t M);
  *   GPU that loads the library 8 MiB + 64 KiB of device memory until exit.
  *   The first call on a device looks up the scratch address for that device
  *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture on the device.
+ *   before any stream capture on the device.  A failed lookup returns
+ *   FP8Q_ERR_CUDA and is not remembered: the next call tries again.
  *   All calls on a device share the one scratch array and nothing in it needs
  *   to start at zero (each call overwrites the codes and scales it reads);
  *   two calls whose work overlaps on the GPU (different streams without

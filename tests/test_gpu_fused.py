@@ -1,6 +1,7 @@
 """GPU parity of the fused quantize + FP8 linear + dequantize path
-(fp8q_quantized_linear): one kernel for up to 16 token rows, the two-step
-path through a caller workspace above that."""
+(fp8q_quantized_linear): one kernel for up to 64 token rows (the CTAs of a
+split-K cluster share the row maxima of their K slices), the two-step path
+through a caller workspace above that."""
 import numpy as np
 import pytest
 import torch
@@ -27,14 +28,18 @@ def oracle(X, W):
     return linear_ref(xq, sx, wq, sw)
 
 
-@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("M", [1, 5, 16, 17, 32, 33, 64])
 @pytest.mark.parametrize("N,K", [(4096, 4096), (264, 272), (1000, 2048), (6144, 2048), (256, 16)])
 def test_fused_against_oracle(fq, M, N, K):
     X = wl.random_f16((M, K), seed=M + N + K, std=2.0)
     W = wl.random_f16((N, K), seed=N * 3 + K, std=0.02)
     Wq, s_w = fq.quantize_weight_per_channel(W.cuda())
     Y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
-    fq.quantized_linear(X.cuda(), Wq, s_w, out=Y, fused=True)
+    # the raw call without a workspace: it must take the one-kernel path
+    Xd = X.cuda()
+    st = _lib.fp8q_quantized_linear(Xd.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K, Y.data_ptr(), 0, 0,
+                                    torch.cuda.current_stream().cuda_stream)
+    assert st == _lib.FP8Q_OK, _lib.last_error_message()
     assert_close_f16(to_np(Y), oracle(X, W), f"fused {M}x{N}x{K}")
     Y2 = fq.quantized_linear(X.cuda(), Wq, s_w)        # two-step through a workspace
     assert_close_f16(to_np(Y2), oracle(X, W), f"two-step {M}x{N}x{K}")
@@ -42,15 +47,19 @@ def test_fused_against_oracle(fq, M, N, K):
 
 
 @pytest.mark.parametrize("ksplit", [1, 2, 4, 8])
-def test_fused_equals_two_step_bitwise(fq, ksplit):
+@pytest.mark.parametrize("M", [7, 40, 64])
+def test_fused_equals_two_step_bitwise(fq, ksplit, M):
     # Same split, same K blocks per CTA: the in-kernel quantization must give
     # exactly the quantizer kernel's codes and scales, hence identical output.
-    M, N, K = 7, 2048, 2048
+    N, K = 2048, 2048
     X = wl.sweep_x(M)[:, :K].contiguous().cuda()
     Wq, s_w = fq.quantize_weight_per_channel(wl.random_f16((N, K), seed=5, std=0.02).cuda())
     fq.set_gemm_tuning(0, 0, ksplit)
     try:
-        Yf = fq.quantized_linear(X, Wq, s_w, fused=True)
+        Yf = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        st = _lib.fp8q_quantized_linear(X.data_ptr(), Wq.data_ptr(), s_w.data_ptr(), M, N, K, Yf.data_ptr(), 0, 0,
+                                        torch.cuda.current_stream().cuda_stream)
+        assert st == _lib.FP8Q_OK, _lib.last_error_message()
         Xq, s_x = fq.quantize_rows_dynamic(X)
         Y2 = fq.linear(Xq, s_x, Wq, s_w)
     finally:

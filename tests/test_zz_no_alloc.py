@@ -43,13 +43,21 @@ def _noalloc(X, Wq, s_w, N):
 
 def test_noalloc_matches_existing_entry_point_twice():
     import fp8_quantized_generative_b200 as fq
-    cases = [(300, 520, 1040, 11), (4096, 6144, 2048, 12)]   # second call reuses the same scratch
+    # Largest first (it fills the scratch exactly: M*K = 8388608 codes), then
+    # smaller shapes that reuse the same scratch, so codes or scales left over
+    # from an earlier, larger call would show up; the last one (8 rows) runs
+    # the split-K kernel, the others the CTA-pair kernel.
+    cases = [(4096, 6144, 2048, 12), (300, 520, 1040, 11), (8, 4096, 4096, 13)]
     for M, N, K, seed in cases:
         X = wl.random_f16((M, K), seed=seed, std=2.0).cuda()
         Wq, s_w = fq.quantize_weight_per_channel(wl.random_f16((N, K), seed=seed + 1, std=0.02).cuda())
-        y_ref = to_np(_existing(X, Wq, s_w, N))
-        y_new = to_np(_noalloc(X, Wq, s_w, N))
-        assert_close_f16(y_new, y_ref, f"noalloc {M}x{N}x{K}")
+        y_ref = _existing(X, Wq, s_w, N)
+        y_new = _noalloc(X, Wq, s_w, N)
+        torch.cuda.synchronize()
+        # the same kernels on the same inputs: bit for bit, and within the
+        # path's tolerance of the oracle-checked entry point
+        assert torch.equal(y_new.view(torch.int16), y_ref.view(torch.int16)), f"noalloc {M}x{N}x{K} not bitwise equal"
+        assert_close_f16(to_np(y_new), to_np(y_ref), f"noalloc {M}x{N}x{K}")
     assert fq.device_error() == 0
 
 
@@ -58,3 +66,6 @@ def test_noalloc_rejects_sizes_beyond_the_scratch():
     st = _lib.fp8q_quantized_linear_noalloc(a, a, a, 4097, 16, 2048, a, 0)   # M*K > 8 Mi
     assert st == _lib.FP8Q_ERR_INVALID_ARG
     assert "8388608" in _lib.last_error_message()
+    st = _lib.fp8q_quantized_linear_noalloc(a, a, a, 16385, 16, 16, a, 0)    # M > 16384 scales
+    assert st == _lib.FP8Q_ERR_INVALID_ARG
+    assert "16384" in _lib.last_error_message()

@@ -11,17 +11,19 @@
 // The weight scale changes every 128 inputs, so one TMEM accumulator cannot
 // carry the whole K loop.  Instead each K block's MMAs (M = 128 token rows,
 // N = 256 weight rows = two scale blocks, four K = 32 instructions) write a
-// fresh FP32 partial into one of two TMEM buffers, and sixteen promotion
-// warps add partial * scale into FP32 accumulators held in registers (each
-// warp: 32 rows x 64 columns, one scale per K block) while the tensor core
-// fills the other buffer.  After the last K block the accumulators are
-// multiplied by s_x and stored as fp16 through swizzled staging tiles and
-// bulk tensor stores (coalesced masked stores where an expert group ends
-// inside a warp's rows).
+// fresh FP32 partial into one of two TMEM buffers, and eight promotion warps
+// add partial * scale into FP32 accumulators held in registers while the
+// tensor core fills the other buffer.  Each promotion warp owns 32 rows (its
+// TMEM lane quadrant) x 128 columns -- exactly one weight scale block, so one
+// scale per K block -- and reads its partial 16 columns at a time with the
+// next load in flight while it multiplies and adds the current one.  After
+// the last K block the accumulators are multiplied by s_x and stored as fp16
+// through two swizzled staging tiles per warp and bulk tensor stores
+// (coalesced masked stores where an expert group ends inside a warp's rows).
 //
 //   warp 0       TMA producer (A = token rows, B = expert weight rows)
 //   warp 1       MMA issuer: K block j -> TMEM partial buffer j % 2
-//   warps 2..17  promotion and epilogue
+//   warps 2..9   promotion and epilogue
 // Tile schedule: the same device-built (expert, n-block, m-block) order as
 // the per-channel grouped kernel (gemm_fp8.cuh).  No TMA multicast.
 #pragma once
@@ -33,7 +35,7 @@ namespace fp8q {
 
 constexpr int kBsBN = 256;                          // tile width (two 128-column scale blocks)
 constexpr int kBsBlk = 128;                         // scale block edge
-constexpr int kBsWarps = 16;                        // promotion warps: 4 per TMEM lane quadrant
+constexpr int kBsWarps = 8;                         // promotion warps: 2 per TMEM lane quadrant
 constexpr int kBsThreads = (kEpiWarp0 + kBsWarps) * 32;
 constexpr int kBsMaxExperts = 128;
 
@@ -42,7 +44,7 @@ struct BsLayout {
   static constexpr int kABytes = kBM * kBK;
   static constexpr int kBBytes = kBsBN * kBK;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kEpiBytes = kBsWarps * kStageTileBytes;
+  static constexpr int kEpiBytes = 2 * kBsWarps * kStageTileBytes;   // two staging tiles per warp
   static constexpr int kNumBars = 2 * STAGES + 5;   // full, empty, pfull[2], pempty[2], drain
   static constexpr int kTmemCols = 2 * kBsBN;       // two partial buffers
   static constexpr int kFixedBytes = STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 32;
@@ -51,8 +53,7 @@ struct BsLayout {
 
 // p.s_w holds the block scales [E, NB, KB] (NB = ceil(N/128), KB = ceil(K/128)).
 template <int STAGES>
-// 18 warps are allocated as 20 (groups of four): at most 96 registers per thread.
-__global__ void __maxnreg__(96)
+__global__ void __launch_bounds__(kBsThreads, 1)
     fp8_gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                                 const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
   using L = BsLayout<STAGES>;
@@ -206,26 +207,26 @@ __global__ void __maxnreg__(96)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ promotion + epilogue
-    const int pw = warp - kEpiWarp0;            // 0..15
+    const int pw = warp - kEpiWarp0;            // 0..7
     const int q = warp & 3;                     // TMEM lane quadrant this warp may read
-    const int c64 = pw >> 2;                    // which 64 of the tile's 256 columns
-    uint8_t* stage = sEpi + pw * kStageTileBytes;
+    const int c128 = pw >> 2;                   // which 128 of the tile's 256 columns (one scale block)
+    uint8_t* stage = sEpi + pw * kStageTileBytes;   // buffer b at + b * kBsWarps * kStageTileBytes
     int pb = 0;
     uint32_t pb_ph = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const TileCoord c = decode_tile<true, BN>(t, p, num_m, num_n, tile_prefix, offs);
       const int e = c.b_row0 / p.N;              // expert of the tile
-      const int nbi = c.n0 / kBsBlk + (c64 >> 1);
+      const int nbi = c.n0 / kBsBlk + c128;
       const float* srow = p.s_w + (static_cast<int64_t>(e) * NB + (nbi < NB ? nbi : 0)) * num_kb;
       const bool cols_live = nbi < NB;
       const int qrow0 = c.a_row0 + q * 32;
       const int valid = c.row_end - qrow0;      // rows of this warp stored (<= 0: none)
       const float sx = lane < valid ? __ldg(p.s_x + qrow0 + lane) : 0.0f;
       float sc = (cols_live && lane < num_kb) ? __ldg(srow + lane) : 0.0f;   // scales of K blocks 0..31
-      float acc[64];
+      float acc[128];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+      for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
       for (int kb = 0; kb < num_kb; ++kb) {
         if (kb > 0 && (kb & 31) == 0) sc = (cols_live && kb + lane < num_kb) ? __ldg(srow + kb + lane) : 0.0f;
         const float s_blk = __shfl_sync(0xffffffffu, sc, kb & 31);
@@ -237,14 +238,16 @@ __global__ void __maxnreg__(96)
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>(pb * BN + c64 * 64);
+                               static_cast<uint32_t>(pb * BN + c128 * 128);
+        // 16 columns at a time, the load of chunk ch+1 in flight during chunk ch
+        uint32_t v[2][16];
+        tmem_ld_32x32b_x16(taddr, v[0]);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {   // 8 columns at a time: the 18 warps fit 96 registers each
-          uint32_t v[8];
-          tmem_ld_32x32b_x8(taddr + static_cast<uint32_t>(ch * 8), v);
-          tmem_ld_wait_regs8(v);
+        for (int ch = 0; ch < 8; ++ch) {
+          tmem_ld_wait_regs16(v[ch & 1]);
+          if (ch + 1 < 8) tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>((ch + 1) * 16), v[(ch + 1) & 1]);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[ch * 8 + i] = fmaf(__uint_as_float(v[i]), s_blk, acc[ch * 8 + i]);
+          for (int i = 0; i < 16; ++i) acc[ch * 16 + i] = fmaf(__uint_as_float(v[ch & 1][i]), s_blk, acc[ch * 16 + i]);
         }
         tc_fence_before();
         __syncwarp();
@@ -253,19 +256,22 @@ __global__ void __maxnreg__(96)
         if (pb == 0) pb_ph ^= 1u;
       }
       if (!ok || valid <= 0) continue;
-      // y = fp16(acc * s_x): two 32 x 32 chunks through the staging tile
+      // y = fp16(acc * s_x): four 32 x 32 chunks through two staging tiles
       const bool bulk = valid >= 32;
-      const uint32_t sbase = smem_u32(stage);
+      // no store of an earlier tile may still read either staging tile
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const int cl = c64 * 64 + ch * 32;      // first column of the chunk within the tile
+      for (int ch = 0; ch < 4; ++ch) {
+        const int cl = c128 * 128 + ch * 32;    // first column of the chunk within the tile
+        const uint32_t sbase = smem_u32(stage + (ch & 1) * kBsWarps * kStageTileBytes);
         uint32_t packed[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const __half2 hv = __floats2half2_rn(__fmul_rn(acc[ch * 32 + 2 * i], sx), __fmul_rn(acc[ch * 32 + 2 * i + 1], sx));
           packed[i] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        if (lane == 0) bulk_wait_read_all();
+        if (lane == 0 && ch >= 2) bulk_wait_read_1();   // the store of chunk ch-2 has read this tile
         __syncwarp();
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4)
@@ -275,7 +281,7 @@ __global__ void __maxnreg__(96)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmY, stage, c.n0 + cl, qrow0);
+            tma_store_2d(&tmY, stage + (ch & 1) * kBsWarps * kStageTileBytes, c.n0 + cl, qrow0);
             bulk_commit_group();
           }
         } else {

@@ -167,6 +167,7 @@ struct Knobs {
   int ksplit = 0; // split-K cluster size, 0 = automatic
   int half_tiles = 1; // FP8Q_HALF_TILES: 0 = CTA-pair grouped kernel uses only M = 256 tiles
   int stage_k = 256;  // FP8Q_STAGE_K: K bytes per stage of the dense pair kernel (128 or 256)
+  int splitk_stage_k = 0;    // FP8Q_SPLITK_STAGE_K: the same for the split-K kernel (0 = by row count)
 };
 Knobs& knobs() {
   static Knobs k = []() {
@@ -180,6 +181,10 @@ Knobs& knobs() {
     if (const char* b = std::getenv("FP8Q_BN")) r.bn = std::atoi(b);
     if (const char* h = std::getenv("FP8Q_HALF_TILES")) r.half_tiles = h[0] == '0' ? 0 : 1;
     if (const char* v = std::getenv("FP8Q_STAGE_K")) r.stage_k = std::atoi(v) == 128 ? 128 : 256;
+    if (const char* v = std::getenv("FP8Q_SPLITK_STAGE_K")) {
+      const int k = std::atoi(v);
+      r.splitk_stage_k = k == 256 ? 256 : k == 128 ? 128 : 0;
+    }
     return r;
   }();
   return k;
@@ -408,16 +413,16 @@ int choose_pair_bn(int64_t M, int64_t N, int clusters) {
 }
 
 // How many clusters of S CTAs of a split-K kernel fit on the device at once.
-template <int MPAD, int STAGES, bool kFused>
+template <int MPAD, int STAGES, bool kFused, int SK = kBK>
 int max_splitk_clusters(int dev, int S) {
   static int cache[kMaxDevices][9] = {};
   static std::mutex mu;
   std::lock_guard<std::mutex> g(mu);
   if (cache[dev][S] != 0) return cache[dev][S];
-  using L = SplitKLayout<MPAD, STAGES, kFused>;
-  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>;
+  using L = SplitKLayout<MPAD, STAGES, kFused, SK>;
+  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES, kFused, SK>;
   const size_t max_smem = kFused ? L::fused_smem_bytes(L::kFusedMaxKBlocks) : L::kSmemBytes;
-  if (ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>>(max_smem, dev) != cudaSuccess) {
+  if (ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES, kFused, SK>>(max_smem, dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return -1;
   }
@@ -447,12 +452,12 @@ int max_splitk_clusters(int dev, int S) {
 // the largest that keeps every cluster of the grid resident at once (one
 // wave; two CTAs share an SM when their shared memory allows) and gives
 // each CTA at least one K block.
-template <int MPAD, int STAGES, bool kFused>
+template <int MPAD, int STAGES, bool kFused, int SK = kBK>
 int choose_ksplit(int dev, int n_tiles, int num_kb) {
   int S = 8;
   while (S > 1 && S > num_kb) S >>= 1;
   while (S > 1) {
-    const int fit = max_splitk_clusters<MPAD, STAGES, kFused>(dev, S);
+    const int fit = max_splitk_clusters<MPAD, STAGES, kFused, SK>(dev, S);
     if (fit >= n_tiles) break;
     S >>= 1;
   }
@@ -462,9 +467,9 @@ int choose_ksplit(int dev, int n_tiles, int num_kb) {
 // Dense linear with at most 128 token rows.  kFused: A is the fp16
 // activations (p.x_f16) and the kernel quantizes them itself (<= 16 rows);
 // otherwise A is Xq with scales s_x.
-template <int MPAD, int STAGES, bool kFused>
+template <int MPAD, int STAGES, bool kFused, int SK = kBK>
 fp8q_status launch_splitk(const uint8_t* Xq, const uint8_t* Wq, const GemmParams& p, int dev, cudaStream_t st) {
-  using L = SplitKLayout<MPAD, STAGES, kFused>;
+  using L = SplitKLayout<MPAD, STAGES, kFused, SK>;
   CUtensorMap tw, tx;
   fp8q_status s = make_operand_map(&tw, Wq, p.N, p.K, kBM);
   if (s != FP8Q_OK) return s;
@@ -475,16 +480,16 @@ fp8q_status launch_splitk(const uint8_t* Xq, const uint8_t* Wq, const GemmParams
     if (s != FP8Q_OK) return s;
   }
   const int n_tiles = (p.N + kBM - 1) / kBM;
-  const int num_kb = (p.K + kBK - 1) / kBK;
-  const int S = knobs().ksplit ? knobs().ksplit : choose_ksplit<MPAD, STAGES, kFused>(dev, n_tiles, num_kb);
+  const int num_kb = (p.K + SK - 1) / SK;
+  const int S = knobs().ksplit ? knobs().ksplit : choose_ksplit<MPAD, STAGES, kFused, SK>(dev, n_tiles, num_kb);
   const int nkb_max = (num_kb + S - 1) / S;
   if (kFused && nkb_max > L::kFusedMaxKBlocks) {
     g_last_error = "fused path: too many K blocks per CTA";
     return FP8Q_ERR_UNSUPPORTED;
   }
   const size_t smem = kFused ? L::fused_smem_bytes(nkb_max) : L::kSmemBytes;
-  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>;
-  cudaError_t e = ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES, kFused>>(
+  auto kernel = fp8_gemm_splitk_kernel<MPAD, STAGES, kFused, SK>;
+  cudaError_t e = ensure_smem<fp8_gemm_splitk_kernel<MPAD, STAGES, kFused, SK>>(
       kFused ? L::fused_smem_bytes(L::kFusedMaxKBlocks) : L::kSmemBytes, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(splitk)");
   e = launch_ex(kernel, dim3(n_tiles * S), dim3(kSkThreads), smem, st, S, true, tw, tx, p);
@@ -501,6 +506,17 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
     // Up to 64 rows the stage count keeps shared memory under half an SM
     // (two CTAs resident), so the CTAs of the next kernel on the stream can
     // start and prefetch their weights while this one drains.
+    // Two 128-byte K boxes per stage above 16 rows (measured on B200: M=64
+    // 9.2 -> 8.1 us, M=32 and M=128 ~2% faster); up to 16 rows one box per
+    // stage, whose five stages prefetch more of the weight slice before the
+    // dependency wait (M=1: 5.7 us against 6.0 us with two-box stages).
+    const int sk = kn.splitk_stage_k ? kn.splitk_stage_k : (p.rows <= 16 ? 128 : 256);
+    if (sk == 256) {
+      if (p.rows <= 16) return launch_splitk<16, 2, false, 256>(Xq, Wq, p, dev, st);
+      if (p.rows <= 32) return launch_splitk<32, 2, false, 256>(Xq, Wq, p, dev, st);
+      if (p.rows <= 64) return launch_splitk<64, 2, false, 256>(Xq, Wq, p, dev, st);
+      if (p.rows <= 128) return launch_splitk<128, 2, false, 256>(Xq, Wq, p, dev, st);
+    }
     if (p.rows <= 16) return launch_splitk<16, 5, false>(Xq, Wq, p, dev, st);
     if (p.rows <= 32) return launch_splitk<32, 4, false>(Xq, Wq, p, dev, st);
     if (p.rows <= 64) return launch_splitk<64, 3, false>(Xq, Wq, p, dev, st);

@@ -44,10 +44,16 @@ constexpr int kSkThreads = 192;   // producer, MMA, 4 epilogue warps
 // codes are made in shared memory), so a stage is a weight tile alone and the
 // CTA stays small enough for two to share an SM (the next kernel's CTAs can
 // then start and stream their weights while this one finishes).
-template <int MPAD, int STAGES, bool kFused = false>
+// SK: K bytes per stage, one 128-byte swizzle box (kBK) per operand or two
+// side by side (2 * kBK: eight MMAs per barrier wait; each mbarrier test in
+// the issuing thread costs ~100 ns while MMAs are in flight).
+template <int MPAD, int STAGES, bool kFused = false, int SK = kBK>
 struct SplitKLayout {
-  static constexpr int kWBytes = kBM * kBK;            // 128 weight rows x 128 K bytes
-  static constexpr int kXBytes = MPAD * kBK;           // MPAD token rows
+  static constexpr int kBoxes = SK / kBK;
+  static constexpr int kWBox = kBM * kBK;
+  static constexpr int kXBox = MPAD * kBK;
+  static constexpr int kWBytes = kBM * SK;             // 128 weight rows x SK K bytes
+  static constexpr int kXBytes = MPAD * SK;            // MPAD token rows
   static constexpr int kStageBytes = kFused ? kWBytes : kWBytes + kXBytes;
   static constexpr int kRingBytes = STAGES * kStageBytes;
   // Partial rows of MPAD + 4 fp32 words (16-byte aligned rows; the +4 keeps
@@ -124,11 +130,12 @@ __device__ __forceinline__ void splitk_reduce_store(const GemmParams& p, const f
   }
 }
 
-template <int MPAD, int STAGES, bool kFused>
+template <int MPAD, int STAGES, bool kFused, int SK = kBK>
 __global__ void __launch_bounds__(kSkThreads, 1)
     fp8_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                            const GemmParams p) {
-  using L = SplitKLayout<MPAD, STAGES, kFused>;
+  using L = SplitKLayout<MPAD, STAGES, kFused, SK>;
+  static_assert(SK == kBK || (SK == 2 * kBK && !kFused), "stage K: one box, or two for the unfused form");
   static_assert(MPAD % 16 == 0 && MPAD >= 16 && MPAD <= 128, "MPAD");
   // swap-AB: B = activations (E4M3, or E5M2 for the variant; the fused path is E4M3)
   const uint32_t kIdesc = idesc_e4m3_f32(kBM, MPAD) | idesc_b_fmt(kFused ? kFmtE4M3 : p.x_fmt);
@@ -160,7 +167,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   const int rank = static_cast<int>(cluster_ctarank());
   const int n_tile = static_cast<int>(blockIdx.x) / S;
   const int n0 = n_tile * kBM;
-  const int num_kb = (p.K + kBK - 1) / kBK;
+  const int num_kb = (p.K + SK - 1) / SK;   // stages of SK bytes of K
   const int kb0 = static_cast<int>((int64_t(rank) * num_kb) / S);
   const int kb1 = static_cast<int>((int64_t(rank + 1) * num_kb) / S);
   const int nkb = kb1 - kb0;
@@ -181,6 +188,17 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   // depend on the kernel launched before this one (programmatic dependent
   // launch), so their DRAM latency overlaps that kernel and this set-up.
   const int pre = nkb < STAGES ? nkb : STAGES;
+  // One stage's weight / activation boxes (kBoxes of 128 bytes of K each).
+  auto load_w = [&](int s, int kb) {
+#pragma unroll
+    for (int j = 0; j < L::kBoxes; ++j)
+      tma_load_2d(sW + s * L::kWBytes + j * L::kWBox, &tmW, &full[s], kb * SK + j * kBK, n0);
+  };
+  auto load_x = [&](int s, int kb) {
+#pragma unroll
+    for (int j = 0; j < L::kBoxes; ++j)
+      tma_load_2d(sX + s * L::kXBytes + j * L::kXBox, &tmX, &full[s], kb * SK + j * kBK, 0);
+  };
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -199,12 +217,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     if (kFused) mbar_arrive_expect_tx(pmax_bar, static_cast<uint32_t>(S - 1) * MPAD * 4);
     for (int i = 0; i < pre; ++i) {
       mbar_arrive_expect_tx(&full[i], kLoadBytes);
-      tma_load_2d(sW + i * L::kWBytes, &tmW, &full[i], (kb0 + i) * kBK, n0);
+      load_w(i, kb0 + i);
     }
     // The rest of this CTA's weight slice goes to L2 now, so the whole
     // stream is in flight from the start.
     if (p.l2_prefetch)
-      for (int kb = kb0 + pre; kb < kb1; ++kb) tma_prefetch_l2_2d(&tmW, kb * kBK, n0);
+      for (int kb = kb0 + pre; kb < kb1; ++kb)
+        for (int j = 0; j < L::kBoxes; ++j) tma_prefetch_l2_2d(&tmW, kb * SK + j * kBK, n0);
     prefetch_tmap(&tmX);
   }
   if (warp == 1) {
@@ -228,7 +247,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       // rows come from the previous kernel.
       if (!kFused) {
         pdl_wait_prior_grid();
-        for (int i = 0; i < pre; ++i) tma_load_2d(sX + i * L::kXBytes, &tmX, &full[i], (kb0 + i) * kBK, 0);
+        for (int i = 0; i < pre; ++i) load_x(i, kb0 + i);
       }
       int s = pre % STAGES;
       uint32_t ph = pre == STAGES ? 1u : 0u;
@@ -240,8 +259,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           break;
         }
         mbar_arrive_expect_tx(&full[s], kLoadBytes);
-        tma_load_2d(sW + s * L::kWBytes, &tmW, &full[s], kb * kBK, n0);
-        if (!kFused) tma_load_2d(sX + s * L::kXBytes, &tmX, &full[s], kb * kBK, 0);
+        load_w(s, kb);
+        if (!kFused) load_x(s, kb);
         armed |= 1u << s;
         armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
         if (++s == STAGES) {
@@ -276,9 +295,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         const uint64_t a0 = sw128_kmajor_desc(smem_u32(sW + s * L::kWBytes));
         const uint64_t b0 = sw128_kmajor_desc(smem_u32(kFused ? fz_codes + kb * L::kXBytes : sX + s * L::kXBytes));
 #pragma unroll
-        for (int k = 0; k < kBK / kUmmaK; ++k)
-          mma_f8f6f4(tmem_base, a0 + static_cast<uint64_t>(k * kUmmaK / 16), b0 + static_cast<uint64_t>(k * kUmmaK / 16),
-                     kIdesc, (kb | k) != 0 ? 1u : 0u);
+        for (int k = 0; k < SK / kUmmaK; ++k) {
+          // box k / 4 of the stage, 32-byte step k % 4 inside its swizzle row
+          const int box = k / (kBK / kUmmaK), kin = k % (kBK / kUmmaK);
+          mma_f8f6f4(tmem_base, a0 + static_cast<uint64_t>(box * (L::kWBox >> 4) + kin * kUmmaK / 16),
+                     b0 + static_cast<uint64_t>(box * (L::kXBox >> 4) + kin * kUmmaK / 16), kIdesc,
+                     (kb | k) != 0 ? 1u : 0u);
+        }
         mma_commit(&empty[s]);
         if (++s == STAGES) {
           s = 0;

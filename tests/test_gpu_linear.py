@@ -161,6 +161,33 @@ def test_splitk_variants(fq, ksplit, M, N, K):
         fq.set_gemm_tuning(0, 0, 0)
 
 
+def test_split_k_stage_forms_in_a_subprocess():
+    # The split-K kernel (M <= 128) runs one-box stages up to 16 rows and
+    # two-box stages above; both forms are forced for every row count here
+    # (FP8Q_SPLITK_STAGE_K is read once per process) and checked against the
+    # oracle, including ragged K and a forced split of 8.
+    import os
+    import subprocess
+    import sys
+    code = r'''
+import sys, torch
+sys.path.insert(0, "tests")
+from test_gpu_linear import check
+import fp8_quantized_generative_b200 as fq
+from fp8_quantized_generative_b200 import workloads as wl
+for M, N, K in [(1, 4096, 4096), (16, 1000, 2048), (33, 520, 1040), (100, 6144, 2048), (128, 264, 272)]:
+    for ks in (0, 8):
+        fq.set_gemm_tuning(3, 0, ks)
+        check(fq, wl.random_f16((M, K), seed=M + K), wl.random_f16((N, K), seed=N, std=0.02), what=f"{M}x{N}x{K} S={ks}")
+print("ok")
+'''
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for sk in ("128", "256"):
+        env = dict(os.environ, FP8Q_SPLITK_STAGE_K=sk)
+        r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0 and r.stdout.strip().endswith("ok"), sk + r.stdout[-2000:] + r.stderr[-2000:]
+
+
 def test_one_box_stages_path_in_a_subprocess():
     # The dense CTA-pair kernel runs 256-byte K stages by default; the
     # one-box (128-byte) stage form stays selectable (FP8Q_STAGE_K=128, read

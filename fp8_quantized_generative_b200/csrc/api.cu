@@ -385,25 +385,35 @@ fp8q_status launch_pair(const uint8_t* A, const uint8_t* B, int64_t b_rows, cons
 }
 
 // Pair-kernel tile width: the candidate with the least modelled time =
-// rounds of tiles (after the tail split) x per-tile work / relative
-// efficiency.  Narrower tiles move more operand bytes out of L2 per FLOP
-// (256 FLOP/B per SM at BN = 256, 219 at 192, 171 at 128) and pay the
-// per-tile epilogue more often; the efficiency factors are per-FLOP
-// throughputs relative to BN = 256 measured on B200 (4096 x 6144 x 2048).
+// rounds of tiles x per-tile work / relative efficiency.  Narrower tiles move
+// more operand bytes out of L2 per FLOP (256 FLOP/B per SM at BN = 256, 219
+// at 192, 171 at 128) and pay the per-tile epilogue more often; the
+// efficiency factors are per-FLOP throughputs relative to BN = 256 measured
+// on B200 (4096 x 6144 x 2048).  Tail pieces (a full tile cut along N for
+// the last round) run at their own width's efficiency, 7% lower still: they
+// keep the full tile's stage layout (measured on B200 at 512 x 4096 x 4096:
+// 128-wide pieces of 256-wide tiles 13.7 us, native 128-wide tiles 12.8 us).
+double pair_tile_efficiency(int width) {
+  return width >= 256 ? 1.0 : width >= 192 ? 0.79 : width >= 128 ? 0.60 : 0.40;
+}
+
 int choose_pair_bn(int64_t M, int64_t N, int clusters) {
   const int cands[3] = {256, 192, 128};
-  const double eff[3] = {1.0, 0.79, 0.60};
+  constexpr double kPiecePenalty = 0.93;
   int best = 256;
   double best_cost = 1e300;
   for (int i = 0; i < 3; ++i) {
     const int bn = cands[i];
     const int64_t full = ((M + 255) / 256) * ((N + bn - 1) / bn);
     const TailSplit ts = tail_split(full, clusters, bn);
-    const int64_t rounds_main = ts.main_tiles / clusters;
-    const int64_t rest = (full - ts.main_tiles) * ts.q;   // pieces after the full rounds
-    const double rounds = static_cast<double>(rounds_main + (ts.main_tiles % clusters ? 1 : 0)) +
-                          static_cast<double>((rest + clusters - 1) / clusters) / ts.q;
-    const double cost = rounds * bn / eff[i];
+    const int64_t rounds_main = (ts.main_tiles + clusters - 1) / clusters;
+    const int64_t pieces = (full - ts.main_tiles) * ts.q;   // after the full rounds
+    const int64_t rounds_tail = (pieces + clusters - 1) / clusters;
+    double cost = static_cast<double>(rounds_main) * bn / pair_tile_efficiency(bn);
+    if (rounds_tail > 0) {
+      const int w = bn / ts.q;
+      cost += static_cast<double>(rounds_tail) * w / (pair_tile_efficiency(w) * (ts.q > 1 ? kPiecePenalty : 1.0));
+    }
     if (cost < best_cost * 0.999) {
       best_cost = cost;
       best = bn;

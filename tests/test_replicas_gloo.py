@@ -53,7 +53,7 @@ def test_reference_arm_runs_only_on_rank_zero(monkeypatch):
     assert bench.run_reference(A, world=2, rank=1) is None
 
 
-@pytest.mark.parametrize("workload", ["tiny", "moe_tokens"])
+@pytest.mark.parametrize("workload", ["tiny", "ffn", "moe_tokens"])
 def test_reference_arm_line_on_rank_zero(workload):
     # the reference arm is the CPU oracle on a bounded sample of the workload;
     # its line carries the contract's keys and a cpu_baseline describing itself

@@ -167,7 +167,7 @@ struct Knobs {
   int ksplit = 0; // split-K cluster size, 0 = automatic
   int half_tiles = 1; // FP8Q_HALF_TILES: 0 = CTA-pair grouped kernel uses only M = 256 tiles
   int stage_k = 256;  // FP8Q_STAGE_K: K bytes per stage of the dense pair kernel (128 or 256)
-  int splitk_stage_k = 0;    // FP8Q_SPLITK_STAGE_K: the same for the split-K kernel (0 = by row count)
+  int splitk_stage_k = 0;    // FP8Q_SPLITK_STAGE_K: the same for the split-K kernel (0 = 256)
 };
 Knobs& knobs() {
   static Knobs k = []() {
@@ -513,20 +513,24 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
   if (e != cudaSuccess) return cuda_fail(e, "device query");
   const Knobs kn = knobs();
   if ((kn.force == 0 && p.rows <= kBM) || kn.force == 3) {
-    // Up to 64 rows the stage count keeps shared memory under half an SM
-    // (two CTAs resident), so the CTAs of the next kernel on the stream can
-    // start and prefetch their weights while this one drains.
-    // Two 128-byte K boxes per stage above 16 rows (measured on B200: M=64
-    // 9.2 -> 8.1 us, M=32 and M=128 ~2% faster); up to 16 rows one box per
-    // stage, whose five stages prefetch more of the weight slice before the
-    // dependency wait (M=1: 5.7 us against 6.0 us with two-box stages).
-    const int sk = kn.splitk_stage_k ? kn.splitk_stage_k : (p.rows <= 16 ? 128 : 256);
+    // Two 128-byte K boxes per stage (eight MMAs per barrier wait), and a
+    // ring deep enough to hold all of a CTA's weight slice at a split of 4
+    // up to 64 rows: the whole slice is requested before the dependency
+    // wait, so it streams in while the kernel before this one (the
+    // activation quantizer) runs.  Measured on B200, quantize + GEMM per
+    // step: M=1 7.9 -> 7.0 us, M=16 8.1 -> 7.5, M=32 9.0 -> 7.9, M=64
+    // 9.8 -> 9.4 against two-stage rings (at M <= 16 the GEMM alone, run
+    // back to back, is ~0.3 us slower: one CTA per SM leaves no room for the
+    // next launch's CTAs).  At 128 rows the partial exchange buffer leaves
+    // room for two stages.
+    const int sk = kn.splitk_stage_k ? kn.splitk_stage_k : 256;
     if (sk == 256) {
-      if (p.rows <= 16) return launch_splitk<16, 2, false, 256>(Xq, Wq, p, dev, st);
-      if (p.rows <= 32) return launch_splitk<32, 2, false, 256>(Xq, Wq, p, dev, st);
-      if (p.rows <= 64) return launch_splitk<64, 2, false, 256>(Xq, Wq, p, dev, st);
+      if (p.rows <= 16) return launch_splitk<16, 4, false, 256>(Xq, Wq, p, dev, st);
+      if (p.rows <= 32) return launch_splitk<32, 4, false, 256>(Xq, Wq, p, dev, st);
+      if (p.rows <= 64) return launch_splitk<64, 3, false, 256>(Xq, Wq, p, dev, st);
       if (p.rows <= 128) return launch_splitk<128, 2, false, 256>(Xq, Wq, p, dev, st);
     }
+    // one-box stages (FP8Q_SPLITK_STAGE_K=128)
     if (p.rows <= 16) return launch_splitk<16, 5, false>(Xq, Wq, p, dev, st);
     if (p.rows <= 32) return launch_splitk<32, 4, false>(Xq, Wq, p, dev, st);
     if (p.rows <= 64) return launch_splitk<64, 3, false>(Xq, Wq, p, dev, st);

@@ -91,8 +91,12 @@ __device__ __forceinline__ void splitk_reduce_store(const GemmParams& p, const f
   const int m4n = (p.rows + 3) >> 2;
   const int items = m4n * NB;
   for (int idx = et; idx < items; idx += 128) {
-    const int nl0 = (idx % NB) * 8;
-    const int m = (idx / NB) * 4;
+    // Token-row blocks vary fastest: the 8 threads of a quarter warp read
+    // one partial row at 8 different 16-byte bank groups (weight rows 8
+    // apart would all map to the same group: 8 x kPitch is a multiple of 32
+    // words).
+    const int m = (idx % m4n) * 4;
+    const int nl0 = (idx / m4n) * 8;
     const int n = n0 + rank * SL + nl0;
     if (n >= p.N) continue;                        // N % 8 == 0: a block is all in or all out
     float acc[8][4];

@@ -162,10 +162,10 @@ def test_splitk_variants(fq, ksplit, M, N, K):
 
 
 def test_split_k_stage_forms_in_a_subprocess():
-    # The split-K kernel (M <= 128) runs one-box stages up to 16 rows and
-    # two-box stages above; both forms are forced for every row count here
-    # (FP8Q_SPLITK_STAGE_K is read once per process) and checked against the
-    # oracle, including ragged K and a forced split of 8.
+    # The split-K kernel (M <= 128) runs two-box (256-byte) stages; the
+    # one-box form stays selectable.  Both are forced for every row count
+    # here (FP8Q_SPLITK_STAGE_K is read once per process) and checked against
+    # the oracle, including ragged K and a forced split of 8.
     import os
     import subprocess
     import sys

@@ -475,7 +475,7 @@ int choose_ksplit(int dev, int n_tiles, int num_kb) {
 }
 
 // Dense linear with at most 128 token rows.  kFused: A is the fp16
-// activations (p.x_f16) and the kernel quantizes them itself (<= 16 rows);
+// activations (p.x_f16) and the kernel quantizes them itself (<= 64 rows);
 // otherwise A is Xq with scales s_x.
 template <int MPAD, int STAGES, bool kFused, int SK = kBK>
 fp8q_status launch_splitk(const uint8_t* Xq, const uint8_t* Wq, const GemmParams& p, int dev, cudaStream_t st) {

@@ -167,7 +167,7 @@ struct Knobs {
   int ksplit = 0; // split-K cluster size, 0 = automatic
   int half_tiles = 1; // FP8Q_HALF_TILES: 0 = CTA-pair grouped kernel uses only M = 256 tiles
   int stage_k = 256;  // FP8Q_STAGE_K: K bytes per stage of the dense pair kernel (128 or 256)
-  int splitk_stage_k = 0;    // FP8Q_SPLITK_STAGE_K: the same for the split-K kernel (0 = 256)
+  int splitk_stage_k = 0;    // FP8Q_SPLITK_STAGE_K: the same for the split-K kernel (0 = 512 up to 32 rows, else 256)
 };
 Knobs& knobs() {
   static Knobs k = []() {
@@ -183,7 +183,7 @@ Knobs& knobs() {
     if (const char* v = std::getenv("FP8Q_STAGE_K")) r.stage_k = std::atoi(v) == 128 ? 128 : 256;
     if (const char* v = std::getenv("FP8Q_SPLITK_STAGE_K")) {
       const int k = std::atoi(v);
-      r.splitk_stage_k = k == 256 ? 256 : k == 128 ? 128 : 0;
+      r.splitk_stage_k = k == 512 ? 512 : k == 256 ? 256 : k == 128 ? 128 : 0;
     }
     return r;
   }();
@@ -513,18 +513,23 @@ fp8q_status launch_dense(const uint8_t* Xq, const uint8_t* Wq, const GemmParams&
   if (e != cudaSuccess) return cuda_fail(e, "device query");
   const Knobs kn = knobs();
   if ((kn.force == 0 && p.rows <= kBM) || kn.force == 3) {
-    // Two 128-byte K boxes per stage (eight MMAs per barrier wait), and a
-    // ring deep enough to hold all of a CTA's weight slice at a split of 4
-    // up to 64 rows: the whole slice is requested before the dependency
-    // wait, so it streams in while the kernel before this one (the
-    // activation quantizer) runs.  Measured on B200, quantize + GEMM per
-    // step: M=1 7.9 -> 7.0 us, M=16 8.1 -> 7.5, M=32 9.0 -> 7.9, M=64
-    // 9.8 -> 9.4 against two-stage rings (at M <= 16 the GEMM alone, run
-    // back to back, is ~0.3 us slower: one CTA per SM leaves no room for the
-    // next launch's CTAs).  At 128 rows the partial exchange buffer leaves
-    // room for two stages.
-    const int sk = kn.splitk_stage_k ? kn.splitk_stage_k : 256;
-    if (sk == 256) {
+    // Several 128-byte K boxes per stage (more MMAs per barrier wait: four
+    // boxes, sixteen MMAs, up to 32 rows; two boxes above, where four would
+    // not leave room for two stages), and a ring deep enough to hold all of
+    // a CTA's weight slice at a split of 4 up to 64 rows: the whole slice is
+    // requested before the dependency wait, so it streams in while the
+    // kernel before this one (the activation quantizer) runs.  Measured on
+    // B200, quantize + GEMM per step: two-box rings of 4 / 4 / 3 stages took
+    // M=1 7.9 -> 7.0 us, M=16 8.1 -> 7.5, M=32 9.0 -> 7.9, M=64 9.8 -> 9.4
+    // against two-stage rings, and four-box stages M=1 7.09 -> 6.78 us,
+    // M=8 7.40 -> 7.06, M=16 7.43 -> 7.11, M=32 7.94 -> 7.70 against those.
+    // At 128 rows the partial exchange buffer leaves room for two stages.
+    const int sk = kn.splitk_stage_k ? kn.splitk_stage_k : (p.rows <= 32 ? 512 : 256);
+    if (sk == 512 && p.rows <= 32) {
+      if (p.rows <= 16) return launch_splitk<16, 2, false, 512>(Xq, Wq, p, dev, st);
+      return launch_splitk<32, 2, false, 512>(Xq, Wq, p, dev, st);
+    }
+    if (sk >= 256) {
       if (p.rows <= 16) return launch_splitk<16, 4, false, 256>(Xq, Wq, p, dev, st);
       if (p.rows <= 32) return launch_splitk<32, 4, false, 256>(Xq, Wq, p, dev, st);
       if (p.rows <= 64) return launch_splitk<64, 3, false, 256>(Xq, Wq, p, dev, st);

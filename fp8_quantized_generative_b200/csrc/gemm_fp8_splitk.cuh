@@ -44,9 +44,10 @@ constexpr int kSkThreads = 192;   // producer, MMA, 4 epilogue warps
 // codes are made in shared memory), so a stage is a weight tile alone and the
 // CTA stays small enough for two to share an SM (the next kernel's CTAs can
 // then start and stream their weights while this one finishes).
-// SK: K bytes per stage, one 128-byte swizzle box (kBK) per operand or two
-// side by side (2 * kBK: eight MMAs per barrier wait; each mbarrier test in
-// the issuing thread costs ~100 ns while MMAs are in flight).
+// SK: K bytes per stage, one 128-byte swizzle box (kBK) per operand, or two
+// or four side by side (2 * kBK / 4 * kBK: eight / sixteen MMAs per barrier
+// wait; each mbarrier test in the issuing thread costs ~100 ns while MMAs
+// are in flight).
 template <int MPAD, int STAGES, bool kFused = false, int SK = kBK>
 struct SplitKLayout {
   static constexpr int kBoxes = SK / kBK;
@@ -139,7 +140,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     fp8_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                            const GemmParams p) {
   using L = SplitKLayout<MPAD, STAGES, kFused, SK>;
-  static_assert(SK == kBK || (SK == 2 * kBK && !kFused), "stage K: one box, or two for the unfused form");
+  static_assert(SK == kBK || ((SK == 2 * kBK || SK == 4 * kBK) && !kFused),
+                "stage K: one box, or two or four for the unfused form");
   static_assert(MPAD % 16 == 0 && MPAD >= 16 && MPAD <= 128, "MPAD");
   // swap-AB: B = activations (E4M3, or E5M2 for the variant; the fused path is E4M3)
   const uint32_t kIdesc = idesc_e4m3_f32(kBM, MPAD) | idesc_b_fmt(kFused ? kFmtE4M3 : p.x_fmt);

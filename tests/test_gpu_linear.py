@@ -162,10 +162,12 @@ def test_splitk_variants(fq, ksplit, M, N, K):
 
 
 def test_split_k_stage_forms_in_a_subprocess():
-    # The split-K kernel (M <= 128) runs two-box (256-byte) stages; the
-    # one-box form stays selectable.  Both are forced for every row count
-    # here (FP8Q_SPLITK_STAGE_K is read once per process) and checked against
-    # the oracle, including ragged K and a forced split of 8.
+    # The split-K kernel (M <= 128) runs four-box (512-byte) stages up to 32
+    # rows and two-box (256-byte) stages above; the one-box form stays
+    # selectable.  Each form is forced for every row count here
+    # (FP8Q_SPLITK_STAGE_K is read once per process; 512 falls back to two
+    # boxes above 32 rows) and checked against the oracle, including ragged
+    # K and a forced split of 8.
     import os
     import subprocess
     import sys
@@ -182,7 +184,7 @@ for M, N, K in [(1, 4096, 4096), (16, 1000, 2048), (33, 520, 1040), (100, 6144, 
 print("ok")
 '''
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    for sk in ("128", "256"):
+    for sk in ("128", "256", "512"):
         env = dict(os.environ, FP8Q_SPLITK_STAGE_K=sk)
         r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True, text=True, timeout=600)
         assert r.returncode == 0 and r.stdout.strip().endswith("ok"), sk + r.stdout[-2000:] + r.stderr[-2000:]

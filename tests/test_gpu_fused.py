@@ -49,9 +49,12 @@ def test_fused_against_oracle(fq, M, N, K):
 @pytest.mark.parametrize("ksplit", [1, 2, 4, 8])
 @pytest.mark.parametrize("M", [7, 40, 64])
 def test_fused_equals_two_step_bitwise(fq, ksplit, M):
-    # Same split, same K blocks per CTA: the in-kernel quantization must give
+    # Same split, same K range per CTA: the in-kernel quantization must give
     # exactly the quantizer kernel's codes and scales, hence identical output.
-    N, K = 2048, 2048
+    # The two paths cut K into stages of different sizes (128 bytes fused,
+    # 256 or 512 bytes for the workspace path), so K is chosen for every CTA
+    # to get whole stages of each: a split of 8 takes K = 4096.
+    N, K = 2048, (4096 if ksplit == 8 else 2048)
     X = wl.sweep_x(M)[:, :K].contiguous().cuda()
     Wq, s_w = fq.quantize_weight_per_channel(wl.random_f16((N, K), seed=5, std=0.02).cuda())
     fq.set_gemm_tuning(0, 0, ksplit)

@@ -352,7 +352,12 @@ fp8q_status fp8q_e4m3_encode_f32(const float* x, int64_t n, uint8_t* out, void* 
  * cluster size 1, 2, 4 or 8 (split-K kernel only).  Process-wide; not thread-safe against
  * concurrent launches.  Environment variables FP8Q_FORCE_KERNEL
  * (auto|single|pair|splitk), FP8Q_BN and FP8Q_KSPLIT (split-K cluster size,
- * 1, 2, 4 or 8) set the initial values.
+ * 1, 2, 4 or 8) set the initial values.  Two more, read once per process,
+ * choose the K bytes a pipeline stage carries (unset: by shape):
+ * FP8Q_STAGE_K = 128 or 256 for the CTA-pair kernel, FP8Q_SPLITK_STAGE_K =
+ * 128, 256 or 512 for the split-K kernel (512 applies up to 32 rows; above,
+ * 256 is used).  Results are the same for every choice up to the order of
+ * the FP32 additions across split-K ranks (which K range each rank takes).
  */
 fp8q_status fp8q_set_gemm_tuning(int kernel_family, int tile_n, int ksplit);
 
